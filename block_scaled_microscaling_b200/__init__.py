@@ -1,0 +1,14 @@
+"""block_scaled_microscaling_b200 -- libmxq, block-scaled shared-exponent
+quantization (AXS-6, MXFP6 E2M3/E3M2, MXFP8 E4M3, MXFP4 E2M1) as hand-written
+CUDA kernels for NVIDIA B200 (sm_100a) behind a C ABI (include/mxq.h).
+
+    from block_scaled_microscaling_b200 import quantize, dequantize, fake_quantize
+    codes, scales = quantize(w_bf16, "mxfp6_e2m3")
+    w2 = dequantize(codes, scales, "mxfp6_e2m3", w_bf16.shape)
+    g_q = fake_quantize(g_fp32, "axs6")          # quantize + dequantize, one pass
+"""
+from .mxq import (EXPORTS, FORMATS, MXQError, dequantize, exp_quantize, fake_quantize, lib, quantize,
+                  quantize_grouped)
+
+__all__ = ["quantize", "dequantize", "fake_quantize", "exp_quantize", "quantize_grouped", "MXQError", "FORMATS",
+           "lib", "EXPORTS"]

@@ -1,0 +1,192 @@
+// mxq_api.cu -- the C ABI of libmxq (declared in include/mxq.h).
+//
+// Host side only: argument validation (before any launch), size queries,
+// status strings, and dispatch to the kernel launchers. Every compute step
+// runs in the kernels of mxq_codec.cu / mxq_expq.cu; there is no host
+// fallback.
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+
+#include "../../include/mxq.h"
+#include "mxq_internal.h"
+
+namespace {
+
+int elem_bits(mxq_format f) {
+    switch (f) {
+        case MXQ_AXS6:
+        case MXQ_MXFP6_E2M3:
+        case MXQ_MXFP6_E3M2: return 6;
+        case MXQ_MXFP8_E4M3: return 8;
+        case MXQ_MXFP4_E2M1: return 4;
+    }
+    return -1;
+}
+bool fmt_ok(mxq_format f) { return elem_bits(f) > 0; }
+bool dtype_ok(mxq_dtype d) { return d == MXQ_F32 || d == MXQ_BF16; }
+int dtype_bytes(mxq_dtype d) { return d == MXQ_F32 ? 4 : 2; }
+
+constexpr int64_t kMaxElems = (int64_t)1 << 50;
+
+mxq_status check_shape(int64_t rows, int64_t cols) {
+    if (rows < 0 || cols <= 0 || cols % 32 != 0) return MXQ_ERR_SHAPE;
+    if (rows > 0 && cols > kMaxElems / rows) return MXQ_ERR_SHAPE;
+    return MXQ_OK;
+}
+
+// device (or managed) memory of the current device, aligned to `align`
+mxq_status check_ptr(const void* p, uintptr_t align) {
+    if (p == nullptr) return MXQ_ERR_INVALID_ARG;
+    cudaPointerAttributes a;
+    cudaError_t e = cudaPointerGetAttributes(&a, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();  // the failed query also sets the (non-sticky) last error: clear it
+        return MXQ_ERR_INVALID_ARG;
+    }
+    if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return MXQ_ERR_INVALID_ARG;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MXQ_ERR_CUDA;
+    if (a.type == cudaMemoryTypeDevice && a.device != dev) return MXQ_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(p) % align != 0) return MXQ_ERR_ALIGN;
+    return MXQ_OK;
+}
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+    uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+size_t codes_bytes(mxq_format f, int64_t rows, int64_t cols) {
+    return (size_t)rows * (size_t)(cols / 32) * (size_t)(4 * elem_bits(f));
+}
+size_t scales_bytes(mxq_format f, int64_t rows, int64_t cols) {
+    return (size_t)rows * (size_t)(cols / 32) * (f == MXQ_AXS6 ? 2u : 1u);
+}
+uintptr_t scales_align(mxq_format f) { return f == MXQ_AXS6 ? 2 : 1; }
+
+mxq_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return MXQ_OK;
+    if (e == cudaErrorNotSupported) return MXQ_ERR_UNSUPPORTED;
+    return MXQ_ERR_CUDA;
+}
+
+#define MXQ_TRY(x)                         \
+    do {                                   \
+        mxq_status s_ = (x);               \
+        if (s_ != MXQ_OK) return s_;       \
+    } while (0)
+
+mxq_status check_quantize_args(mxq_format fmt, const void* src, mxq_dtype dtype, int64_t rows, int64_t cols,
+                               void* codes, void* scales) {
+    if (!fmt_ok(fmt) || !dtype_ok(dtype)) return MXQ_ERR_INVALID_ARG;
+    MXQ_TRY(check_shape(rows, cols));
+    if (rows == 0) return MXQ_OK;
+    MXQ_TRY(check_ptr(src, 16));
+    MXQ_TRY(check_ptr(codes, 16));
+    MXQ_TRY(check_ptr(scales, scales_align(fmt)));
+    const size_t nsrc = (size_t)rows * (size_t)cols * dtype_bytes(dtype);
+    const size_t nc = codes_bytes(fmt, rows, cols), ns = scales_bytes(fmt, rows, cols);
+    if (overlap(src, nsrc, codes, nc) || overlap(src, nsrc, scales, ns) || overlap(codes, nc, scales, ns))
+        return MXQ_ERR_INVALID_ARG;
+    return MXQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mxq_status mxq_quantize(mxq_format fmt, const void* src, mxq_dtype dtype, int64_t rows, int64_t cols, void* codes,
+                        void* scales, mxq_stream stream) {
+    MXQ_TRY(check_quantize_args(fmt, src, dtype, rows, cols, codes, scales));
+    if (rows == 0) return MXQ_OK;
+    mxq::SegTable<1> tab{};
+    tab.seg[0] = {src, codes, scales, rows * (cols / 32), 0};
+    tab.n = 1;
+    return from_cuda(mxq::launch_quantize<1>((int)fmt, (int)dtype, tab, (cudaStream_t)stream));
+}
+
+mxq_status mxq_quantize_grouped(mxq_format fmt, mxq_dtype dtype, const mxq_tensor* tensors, int n,
+                                mxq_stream stream) {
+    if (!fmt_ok(fmt) || !dtype_ok(dtype) || tensors == nullptr || n < 1 || n > MXQ_MAX_GROUP)
+        return MXQ_ERR_INVALID_ARG;
+    mxq::SegTable<mxq::kMaxSeg> tab{};
+    int m = 0;
+    for (int i = 0; i < n; ++i) {
+        const mxq_tensor& t = tensors[i];
+        MXQ_TRY(check_quantize_args(fmt, t.src, dtype, t.rows, t.cols, t.codes, t.scales));
+        if (t.rows == 0) continue;
+        tab.seg[m++] = {t.src, t.codes, t.scales, t.rows * (t.cols / 32), 0};
+    }
+    if (m == 0) return MXQ_OK;
+    tab.n = m;
+    return from_cuda(mxq::launch_quantize<mxq::kMaxSeg>((int)fmt, (int)dtype, tab, (cudaStream_t)stream));
+}
+
+mxq_status mxq_dequantize(mxq_format fmt, const void* codes, const void* scales, int64_t rows, int64_t cols,
+                          void* dst, mxq_dtype dtype, mxq_stream stream) {
+    if (!fmt_ok(fmt) || !dtype_ok(dtype)) return MXQ_ERR_INVALID_ARG;
+    MXQ_TRY(check_shape(rows, cols));
+    if (rows == 0) return MXQ_OK;
+    MXQ_TRY(check_ptr(codes, 16));
+    MXQ_TRY(check_ptr(scales, scales_align(fmt)));
+    MXQ_TRY(check_ptr(dst, 16));
+    const size_t nd = (size_t)rows * (size_t)cols * dtype_bytes(dtype);
+    if (overlap(dst, nd, codes, codes_bytes(fmt, rows, cols)) || overlap(dst, nd, scales, scales_bytes(fmt, rows, cols)))
+        return MXQ_ERR_INVALID_ARG;
+    return from_cuda(mxq::launch_dequantize((int)fmt, codes, scales, dst, (int)dtype, rows * (cols / 32),
+                                            (cudaStream_t)stream));
+}
+
+mxq_status mxq_fake_quantize(mxq_format fmt, const void* src, mxq_dtype dtype, int64_t rows, int64_t cols, void* dst,
+                             mxq_stream stream) {
+    if (!fmt_ok(fmt) || !dtype_ok(dtype)) return MXQ_ERR_INVALID_ARG;
+    MXQ_TRY(check_shape(rows, cols));
+    if (rows == 0) return MXQ_OK;
+    MXQ_TRY(check_ptr(src, 16));
+    MXQ_TRY(check_ptr(dst, 16));
+    const size_t nb = (size_t)rows * (size_t)cols * dtype_bytes(dtype);
+    if (src != dst && overlap(src, nb, dst, nb)) return MXQ_ERR_INVALID_ARG;
+    return from_cuda(mxq::launch_fake_quantize((int)fmt, src, dst, (int)dtype, rows * (cols / 32),
+                                               (cudaStream_t)stream));
+}
+
+mxq_status mxq_exp_quantize(mxq_format fmt, const float* scores, int64_t rows, int64_t cols, void* codes,
+                            void* scales, mxq_stream stream) {
+    MXQ_TRY(check_quantize_args(fmt, scores, MXQ_F32, rows, cols, codes, scales));
+    if (!mxq::exp_quantize_supported(cols)) return MXQ_ERR_UNSUPPORTED;
+    if (rows == 0) return MXQ_OK;
+    return from_cuda(mxq::launch_exp_quantize((int)fmt, scores, rows, cols, codes, scales, (cudaStream_t)stream));
+}
+
+size_t mxq_codes_bytes(mxq_format fmt, int64_t rows, int64_t cols) {
+    if (!fmt_ok(fmt) || check_shape(rows, cols) != MXQ_OK) return 0;
+    return codes_bytes(fmt, rows, cols);
+}
+
+size_t mxq_scales_bytes(mxq_format fmt, int64_t rows, int64_t cols) {
+    if (!fmt_ok(fmt) || check_shape(rows, cols) != MXQ_OK) return 0;
+    return scales_bytes(fmt, rows, cols);
+}
+
+int mxq_block_bits(mxq_format fmt) {
+    if (!fmt_ok(fmt)) return -1;
+    return 8 + 32 * elem_bits(fmt) + (fmt == MXQ_AXS6 ? 2 : 0);
+}
+
+const char* mxq_status_string(mxq_status s) {
+    switch (s) {
+        case MXQ_OK: return "ok";
+        case MXQ_ERR_INVALID_ARG: return "invalid argument (format, type, or a null/host/other-device/overlapping pointer)";
+        case MXQ_ERR_SHAPE: return "invalid shape (rows < 0, cols <= 0, cols not a multiple of 32, or too large)";
+        case MXQ_ERR_ALIGN: return "misaligned pointer (values and codes need 16 bytes, AXS-6 headers 2)";
+        case MXQ_ERR_UNSUPPORTED: return "valid request that this build does not support";
+        case MXQ_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+        case MXQ_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    }
+    return "unknown status";
+}
+
+const char* mxq_version(void) { return "0.1.0"; }
+
+}  // extern "C"

@@ -1,0 +1,195 @@
+// mxq_device.cuh -- device-side building blocks of libmxq (sm_100a).
+//
+// Element formats and the block rule (see include/mxq.h):
+//   "AXS-6: Adaptive eXponent Sharing", block figure -- 8-bit shared exponent
+//   per 32 values, sign + 5-bit magnitude per value (read as m/16);
+//   "Sonar: Online MXFP6", Start a model -- packed six-bit E2M3/E3M2 codes with
+//   an E8M0 scale per block of 32; "EFQ-Softmax", Jargon -- E2M1 (MXFP4),
+//   exponent-only scale from the block's local maximum.
+//
+// Rounding uses the sm_100a conversion instructions
+// cvt.rn.satfinite.{e2m3x2,e3m2x2,e4m3x2,e2m1x2}.f32 (round to nearest even,
+// saturate to the largest finite value), two values per instruction; AXS-6
+// rounds with a float add of 1.5*2^23. Decoding places the magnitude bits
+// into an fp32 bit pattern and rescales by exact powers of two.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace mxq {
+
+enum : int { F_AXS6 = 0, F_E2M3 = 1, F_E3M2 = 2, F_E4M3 = 3, F_E2M1 = 4 };
+
+template <int F> struct Fmt;
+// W: code bits; EMAX: floor(log2 max); M: mantissa bits; BIAS: exponent bias
+template <> struct Fmt<F_AXS6> { static constexpr int W = 6, EMAX = 0, M = 5, BIAS = 0; static constexpr bool FIXED = true; };
+template <> struct Fmt<F_E2M3> { static constexpr int W = 6, EMAX = 2, M = 3, BIAS = 1; static constexpr bool FIXED = false; };
+template <> struct Fmt<F_E3M2> { static constexpr int W = 6, EMAX = 4, M = 2, BIAS = 3; static constexpr bool FIXED = false; };
+template <> struct Fmt<F_E4M3> { static constexpr int W = 8, EMAX = 8, M = 3, BIAS = 7; static constexpr bool FIXED = false; };
+template <> struct Fmt<F_E2M1> { static constexpr int W = 4, EMAX = 2, M = 1, BIAS = 1; static constexpr bool FIXED = false; };
+
+// bytes of one block's packed payload
+template <int F> __host__ __device__ constexpr int payload() { return 4 * Fmt<F>::W; }
+
+// ---------------------------------------------------------------------------
+// memory primitives
+
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+__device__ __forceinline__ void st_stream_v4(void* p, uint4 v) {
+    asm volatile("st.global.L1::no_allocate.v4.u32 [%0], {%1,%2,%3,%4};"
+                 :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// packed fp32 pair arithmetic (one instruction for two IEEE round-to-nearest ops)
+
+__device__ __forceinline__ unsigned long long pk(float a, float b) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1,%2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void upk(unsigned long long r, float& a, float& b) {
+    asm("mov.b64 {%0,%1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ void mul2(float& a, float& b, float s) {
+    unsigned long long r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a, b)), "l"(pk(s, s)));
+    upk(r, a, b);
+}
+
+// ---------------------------------------------------------------------------
+// the shared scale
+
+// |x| bit patterns order as unsigned integers: finite < +Inf < NaN.
+// byte = 0xFF for a NaN/Inf block, else clamp(floor(log2 amax) - EMAX + 127, 0, 254);
+// for amax normal that is max(biased exponent - EMAX, 0), and every subnormal
+// or zero amax gives 0.
+template <int F>
+__device__ __forceinline__ uint32_t scale_byte(uint32_t amax_bits) {
+    int b = (int)(amax_bits >> 23) - Fmt<F>::EMAX;
+    return amax_bits >= 0x7F800000u ? 0xFFu : (uint32_t)max(b, 0);
+}
+
+// 2^(127 - byte) as fp32 (the reciprocal of the block scale), byte in [0, 254]
+__device__ __forceinline__ float inv_scale(uint32_t byte) {
+    uint32_t bits = byte >= 254u ? 0x00400000u : (254u - byte) << 23;
+    return __uint_as_float(bits);
+}
+// 2^(byte - 127) as fp32, byte in [0, 254]
+__device__ __forceinline__ float fwd_scale(uint32_t byte) {
+    return __uint_as_float(byte == 0u ? 0x00400000u : byte << 23);
+}
+
+// ---------------------------------------------------------------------------
+// hardware rounding to the element formats, two at a time: result holds
+// code(lo) in the low byte (low nibble for E2M1) and code(hi) above it.
+
+template <int F> __device__ __forceinline__ uint32_t cvt2(float lo, float hi);
+template <> __device__ __forceinline__ uint32_t cvt2<F_E2M3>(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e2m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+template <> __device__ __forceinline__ uint32_t cvt2<F_E3M2>(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e3m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+template <> __device__ __forceinline__ uint32_t cvt2<F_E4M3>(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+template <> __device__ __forceinline__ uint32_t cvt2<F_E2M1>(float lo, float hi) {
+    uint32_t r;
+    asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u32.u8 %0, t; }"
+        : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// AXS-6 code of x (already multiplied by 2^-Es): sign | min(rne(16|x|), 31).
+// rne by adding 1.5*2^23 (|16x| < 2^22): the sum's low mantissa bits are the
+// rounded integer.
+__device__ __forceinline__ uint32_t axs6_code(float y) {
+    float t = fabsf(y) * 16.0f;
+    uint32_t m = __float_as_uint(t + 12582912.0f) - 0x4B400000u;
+    m = min(m, 31u);
+    return m | ((__float_as_uint(y) >> 26) & 0x20u);
+}
+
+// Codes of n = 2k values, one code per byte (E2M1: one per nibble, packed).
+// Returned as words with codes in ascending byte order.
+//   6-bit / 8-bit formats: out[j] holds codes 4j..4j+3, one per byte.
+//   E2M1: out[j] holds codes 8j..8j+7, one per nibble.
+template <int F, int N>
+__device__ __forceinline__ void encode(const float* y, uint32_t* out) {
+    if constexpr (F == F_AXS6) {
+#pragma unroll
+        for (int j = 0; j < N / 4; ++j)
+            out[j] = axs6_code(y[4 * j]) | axs6_code(y[4 * j + 1]) << 8 | axs6_code(y[4 * j + 2]) << 16 |
+                     axs6_code(y[4 * j + 3]) << 24;
+    } else if constexpr (F == F_E2M1) {
+#pragma unroll
+        for (int j = 0; j < (N + 7) / 8; ++j) {
+            uint32_t w = 0;
+#pragma unroll
+            for (int k = 0; k < 4 && 8 * j + 2 * k < N; ++k) w |= cvt2<F>(y[8 * j + 2 * k], y[8 * j + 2 * k + 1]) << (8 * k);
+            out[j] = w;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < N / 4; ++j)
+            out[j] = cvt2<F>(y[4 * j], y[4 * j + 1]) | cvt2<F>(y[4 * j + 2], y[4 * j + 3]) << 16;
+    }
+}
+
+// four 6-bit codes, one per byte (b0..b3) -> 24-bit field b0 | b1<<6 | b2<<12 | b3<<18
+__device__ __forceinline__ uint32_t pack6x4(uint32_t x) {
+    uint32_t y = (x & 0x003F003Fu) | ((x >> 2) & 0x0FC00FC0u);
+    return (y & 0x00000FFFu) | ((y >> 4) & 0x00FFF000u);
+}
+// inverse: 24-bit field -> four codes, one per byte
+__device__ __forceinline__ uint32_t unpack6x4(uint32_t z) {
+    uint32_t y = (z & 0x00000FFFu) | ((z << 4) & 0x0FFF0000u);
+    return (y & 0x003F003Fu) | ((y << 2) & 0x3F003F00u);
+}
+
+// ---------------------------------------------------------------------------
+// decoding: code -> exact value * 2^(byte-127)
+
+// fp32 bit pattern whose value is decode(code) * 2^-(127-BIAS) (FP formats) or
+// decode(code) * 2^-126 (AXS-6): the magnitude field lands on the fp32
+// exponent/mantissa fields (subnormal patterns included), sign on bit 31.
+template <int F>
+__device__ __forceinline__ uint32_t code_to_bits(uint32_t c) {
+    constexpr int W = Fmt<F>::W;
+    constexpr int SH = Fmt<F>::FIXED ? 19 : 23 - Fmt<F>::M;
+    return ((c & ((1u << (W - 1)) - 1u)) << SH) | ((c << (32 - W)) & 0x80000000u);
+}
+template <int F> __device__ __forceinline__ float decode_unit() {
+    return __uint_as_float((uint32_t)((Fmt<F>::FIXED ? 126 : 127 - Fmt<F>::BIAS) + 127) << 23);
+}
+
+// values of two codes times the block scale s = 2^(byte-127); exact products
+// except for the final rounding of results below the fp32 normal range.
+template <int F>
+__device__ __forceinline__ void decode2(uint32_t c0, uint32_t c1, float s, float& v0, float& v1) {
+    v0 = __uint_as_float(code_to_bits<F>(c0));
+    v1 = __uint_as_float(code_to_bits<F>(c1));
+    mul2(v0, v1, decode_unit<F>());
+    mul2(v0, v1, s);
+}
+
+// fp32 pair -> bf16x2, round to nearest even
+__device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+}  // namespace mxq

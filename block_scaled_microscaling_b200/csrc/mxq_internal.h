@@ -1,0 +1,37 @@
+// mxq_internal.h -- launch interface between the C ABI (mxq_api.cu) and the
+// kernels (mxq_codec.cu, mxq_expq.cu). Not part of the public header.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace mxq {
+
+constexpr int kMaxSeg = 64;  // == MXQ_MAX_GROUP
+
+// one tensor of a (grouped) quantize launch
+struct Seg {
+    const void* src;
+    void* codes;
+    void* scales;
+    long long nblocks;  // blocks of 32 values
+    long long tile0;    // first warp tile of this tensor (filled by the launcher)
+};
+template <int N> struct SegTable {
+    Seg seg[N];
+    int n;
+    long long ntiles;
+};
+
+// fmt: 0 AXS-6, 1 E2M3, 2 E3M2, 3 E4M3, 4 E2M1; dtype: 0 fp32, 1 bf16
+template <int NSEG>
+cudaError_t launch_quantize(int fmt, int dtype, SegTable<NSEG>& tab, cudaStream_t st);
+cudaError_t launch_dequantize(int fmt, const void* codes, const void* scales, void* dst, int dtype,
+                              long long nblocks, cudaStream_t st);
+cudaError_t launch_fake_quantize(int fmt, const void* src, void* dst, int dtype, long long nblocks,
+                                 cudaStream_t st);
+// returns cudaErrorNotSupported when cols is beyond what one cluster holds
+cudaError_t launch_exp_quantize(int fmt, const float* scores, long long rows, long long cols, void* codes,
+                                void* scales, cudaStream_t st);
+bool exp_quantize_supported(long long cols);
+
+}  // namespace mxq

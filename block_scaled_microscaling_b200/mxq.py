@@ -1,0 +1,252 @@
+"""Python binding of libmxq (include/mxq.h), argument marshalling only.
+
+The functions named like the C entry points (mxq_quantize, ...) take raw
+integers (device pointers, sizes, a cudaStream_t handle) and return the
+mxq_status code. The torch-facing helpers below them (quantize, dequantize,
+fake_quantize, exp_quantize, quantize_grouped) only allocate outputs with
+torch, read pointers/strides and the current stream, call the C entry point
+and raise MXQError on a non-zero status. Every step of the method runs in the
+CUDA kernels of libmxq; there is no CPU path: if libmxq.so is missing, every
+call raises.
+"""
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmxq.so")
+
+FORMATS = {"axs6": 0, "mxfp6_e2m3": 1, "mxfp6_e3m2": 2, "mxfp8": 3, "mxfp4": 4}
+DTYPES = {"f32": 0, "bf16": 1}
+STATUS = {0: "MXQ_OK", 1: "MXQ_ERR_INVALID_ARG", 2: "MXQ_ERR_SHAPE", 3: "MXQ_ERR_ALIGN",
+          4: "MXQ_ERR_UNSUPPORTED", 5: "MXQ_ERR_CUDA", 6: "MXQ_ERR_TIMEOUT"}
+MAX_GROUP = 64
+ELEM_BITS = {"axs6": 6, "mxfp6_e2m3": 6, "mxfp6_e3m2": 6, "mxfp8": 8, "mxfp4": 4}
+
+EXPORTS = ["mxq_quantize", "mxq_dequantize", "mxq_fake_quantize", "mxq_exp_quantize", "mxq_quantize_grouped",
+           "mxq_codes_bytes", "mxq_scales_bytes", "mxq_block_bits", "mxq_status_string", "mxq_version"]
+
+
+class MXQError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({mxq_status_string(status)})")
+
+
+class _Tensor(ctypes.Structure):
+    _fields_ = [("src", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libmxq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m block_scaled_microscaling_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        i32, i64, vp, sz = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
+        for name, args in [
+            ("mxq_quantize", [i32, vp, i32, i64, i64, vp, vp, vp]),
+            ("mxq_dequantize", [i32, vp, vp, i64, i64, vp, i32, vp]),
+            ("mxq_fake_quantize", [i32, vp, i32, i64, i64, vp, vp]),
+            ("mxq_exp_quantize", [i32, vp, i64, i64, vp, vp, vp]),
+            ("mxq_quantize_grouped", [i32, i32, ctypes.POINTER(_Tensor), i32, vp]),
+        ]:
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = i32
+        L.mxq_codes_bytes.argtypes = [i32, i64, i64]
+        L.mxq_codes_bytes.restype = sz
+        L.mxq_scales_bytes.argtypes = [i32, i64, i64]
+        L.mxq_scales_bytes.restype = sz
+        L.mxq_block_bits.argtypes = [i32]
+        L.mxq_block_bits.restype = i32
+        L.mxq_status_string.argtypes = [i32]
+        L.mxq_status_string.restype = ctypes.c_char_p
+        L.mxq_version.argtypes = []
+        L.mxq_version.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+# ---- the C entry points, same names and arguments --------------------------------
+
+def mxq_quantize(fmt, src, dtype, rows, cols, codes, scales, stream):
+    return lib().mxq_quantize(fmt, src, dtype, rows, cols, codes, scales, stream)
+
+
+def mxq_dequantize(fmt, codes, scales, rows, cols, dst, dtype, stream):
+    return lib().mxq_dequantize(fmt, codes, scales, rows, cols, dst, dtype, stream)
+
+
+def mxq_fake_quantize(fmt, src, dtype, rows, cols, dst, stream):
+    return lib().mxq_fake_quantize(fmt, src, dtype, rows, cols, dst, stream)
+
+
+def mxq_exp_quantize(fmt, scores, rows, cols, codes, scales, stream):
+    return lib().mxq_exp_quantize(fmt, scores, rows, cols, codes, scales, stream)
+
+
+def mxq_quantize_grouped(fmt, dtype, tensors, stream):
+    """tensors: sequence of (src, codes, scales, rows, cols) integer tuples."""
+    arr = (_Tensor * max(1, len(tensors)))()
+    for i, (s, c, sc, r, k) in enumerate(tensors):
+        arr[i] = _Tensor(s, c, sc, r, k)
+    return lib().mxq_quantize_grouped(fmt, dtype, arr, len(tensors), stream)
+
+
+def mxq_codes_bytes(fmt, rows, cols):
+    return lib().mxq_codes_bytes(fmt, rows, cols)
+
+
+def mxq_scales_bytes(fmt, rows, cols):
+    return lib().mxq_scales_bytes(fmt, rows, cols)
+
+
+def mxq_block_bits(fmt):
+    return lib().mxq_block_bits(fmt)
+
+
+def mxq_status_string(status):
+    return lib().mxq_status_string(status).decode()
+
+
+def mxq_version():
+    return lib().mxq_version().decode()
+
+
+# ---- torch helpers ---------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _fmt(fmt):
+    if fmt not in FORMATS:
+        raise ValueError(f"unknown format {fmt!r}; one of {sorted(FORMATS)}")
+    return FORMATS[fmt]
+
+
+def _dt(t):
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return DTYPES["f32"]
+    if t.dtype == torch.bfloat16:
+        return DTYPES["bf16"]
+    raise TypeError(f"values must be float32 or bfloat16, got {t.dtype}")
+
+
+def _stream(stream):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _as2d(t):
+    if t.dim() == 0:
+        raise ValueError("need at least one dimension")
+    cols = t.shape[-1]
+    rows = t.numel() // cols if cols else 0
+    return rows, cols
+
+
+def _check(status, what):
+    if status != 0:
+        raise MXQError(status, what)
+
+
+def scale_dtype(fmt):
+    torch = _torch()
+    return torch.int16 if fmt == "axs6" else torch.uint8
+
+
+def empty_codes(fmt, rows, cols, device):
+    torch = _torch()
+    return torch.empty((rows, (cols // 32) * 4 * ELEM_BITS[fmt]), dtype=torch.uint8, device=device)
+
+
+def empty_scales(fmt, rows, cols, device):
+    torch = _torch()
+    return torch.empty((rows, cols // 32), dtype=scale_dtype(fmt), device=device)
+
+
+def quantize(x, fmt, codes=None, scales=None, stream=None):
+    """x [..., cols] (bf16/fp32, contiguous, CUDA) -> (codes uint8 [rows, cols/32*P], scales)."""
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    rows, cols = _as2d(x)
+    if codes is None:
+        codes = empty_codes(fmt, rows, cols, x.device)
+    if scales is None:
+        scales = empty_scales(fmt, rows, cols, x.device)
+    _check(mxq_quantize(_fmt(fmt), x.data_ptr(), _dt(x), rows, cols, codes.data_ptr(), scales.data_ptr(),
+                        _stream(stream)), "mxq_quantize")
+    return codes, scales
+
+
+def dequantize(codes, scales, fmt, shape, dtype=None, out=None, stream=None):
+    """codes + scales -> values of `shape` (last dim = cols) and `dtype` (default bf16)."""
+    torch = _torch()
+    if out is None:
+        out = torch.empty(tuple(shape), dtype=dtype or torch.bfloat16, device=codes.device)
+    rows, cols = _as2d(out)
+    _check(mxq_dequantize(_fmt(fmt), codes.data_ptr(), scales.data_ptr(), rows, cols, out.data_ptr(), _dt(out),
+                          _stream(stream)), "mxq_dequantize")
+    return out
+
+
+def fake_quantize(x, fmt="axs6", block_size=32, out=None, stream=None):
+    """Quantize then dequantize in one pass; out=x runs in place."""
+    if block_size != 32:
+        raise MXQError(4, f"block_size={block_size}")
+    torch = _torch()
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    if out is None:
+        out = torch.empty_like(x)
+    rows, cols = _as2d(x)
+    _check(mxq_fake_quantize(_fmt(fmt), x.data_ptr(), _dt(x), rows, cols, out.data_ptr(), _stream(stream)),
+           "mxq_fake_quantize")
+    return out
+
+
+def exp_quantize(scores, fmt="mxfp4", codes=None, scales=None, stream=None):
+    """fp32 scores [..., keys] -> codes + scales of exp(s - rowmax), block-quantized per 32 keys."""
+    torch = _torch()
+    if scores.dtype != torch.float32 or not scores.is_contiguous():
+        raise ValueError("scores must be contiguous float32")
+    rows, cols = _as2d(scores)
+    if codes is None:
+        codes = empty_codes(fmt, rows, cols, scores.device)
+    if scales is None:
+        scales = empty_scales(fmt, rows, cols, scores.device)
+    _check(mxq_exp_quantize(_fmt(fmt), scores.data_ptr(), rows, cols, codes.data_ptr(), scales.data_ptr(),
+                            _stream(stream)), "mxq_exp_quantize")
+    return codes, scales
+
+
+def quantize_grouped(xs, fmt, outs=None, stream=None):
+    """Quantize several tensors of one dtype in one launch; returns [(codes, scales), ...]."""
+    if not xs:
+        return []
+    if len(xs) > MAX_GROUP:
+        raise ValueError(f"at most {MAX_GROUP} tensors per grouped launch")
+    dt = _dt(xs[0])
+    if outs is None:
+        outs = []
+        for x in xs:
+            r, c = _as2d(x)
+            outs.append((empty_codes(fmt, r, c, x.device), empty_scales(fmt, r, c, x.device)))
+    descs = []
+    for x, (c, s) in zip(xs, outs):
+        if _dt(x) != dt or not x.is_contiguous():
+            raise ValueError("grouped tensors must be contiguous and share one dtype")
+        r, k = _as2d(x)
+        descs.append((x.data_ptr(), c.data_ptr(), s.data_ptr(), r, k))
+    _check(mxq_quantize_grouped(_fmt(fmt), dt, descs, _stream(stream)), "mxq_quantize_grouped")
+    return outs

@@ -1,0 +1,179 @@
+/*
+ * mxq.h -- C ABI of libmxq: block-scaled shared-exponent quantization on
+ * NVIDIA B200 (sm_100a).
+ *
+ * A tensor of shape [rows, cols] (row-major, contiguous, cols % 32 == 0) is
+ * cut into blocks of 32 consecutive values along the last dimension. Each
+ * block gets one power-of-two scale 2^Es with
+ *     Es = clamp(floor(log2(max_i |x_i|)) - emax, -127, 127)
+ * stored as an E8M0 byte Es + 127, and every value is rounded to the element
+ * format (round to nearest, ties to even, saturating at the largest finite
+ * magnitude) and bit-packed.
+ *   - "AXS-6: Adaptive eXponent Sharing", block figure: 8-bit shared exponent
+ *     and 2-bit config once per 32 values, sign + 5-bit mantissa per value.
+ *   - "Sonar: Online MXFP6", Start a model / Select the FP6 encoding: packed
+ *     six-bit E2M3 or E3M2 data with an E8M0 scale per block of 32 values.
+ *   - "EFQ-Softmax" explainer, Jargon and stage table: E2M1 (MXFP4) codes, an
+ *     exponent-only block scale taken from the block's local maximum; the
+ *     exp-then-quantize probability stage.
+ *   - "eXmY" abstract: non-power-of-two widths packed densely, byte addressable.
+ *
+ * Element formats (emax = floor(log2 of the largest finite magnitude)):
+ *   MXQ_AXS6        6 bits: sign + 5-bit magnitude m, value m/16;   emax 0, max 31/16
+ *   MXQ_MXFP6_E2M3  6 bits: 1-2-3, bias 1;                           emax 2, max 7.5
+ *   MXQ_MXFP6_E3M2  6 bits: 1-3-2, bias 3;                           emax 4, max 28
+ *   MXQ_MXFP8_E4M3  8 bits: 1-4-3, bias 7, magnitude 0x7F is NaN;    emax 8, max 448
+ *   MXQ_MXFP4_E2M1  4 bits: 1-2-1, bias 1;                           emax 2, max 6
+ * Subnormals (exponent field 0) are value 2^(1-bias) * m / 2^M.
+ *
+ * Memory layouts (all row-major, all owned by the caller):
+ *   values  [rows, cols] fp32 or bf16.
+ *   codes   uint8[rows * cols/32 * P]: block b's payload occupies bytes
+ *           [b*P, (b+1)*P), P = 24 (6-bit formats), 32 (E4M3), 16 (E2M1).
+ *           Inside a payload, value j of the block is bits [w*j, w*j + w) of
+ *           the little-endian bit string (bit k = bit k%8 of byte k/8).
+ *   scales  uint8[rows * cols/32] E8M0 bytes (2^(byte-127); 0xFF = NaN block),
+ *           or for AXS-6 uint16[rows * cols/32] headers: bits 0-7 the shared
+ *           exponent byte, bits 8-9 the config field (written as 0, ignored on
+ *           read), bits 10-15 zero.
+ *
+ * Special values: a block holding a NaN or an infinity gets scale 0xFF and
+ * all-zero codes, and dequantizes to NaN. An all-zero block gets scale 0.
+ * The code's sign bit is the input's sign bit (-0 stays -0). Any NaN that a
+ * dequantize / fake-quantize writes is the canonical quiet NaN (fp32
+ * 0x7FC00000, bf16 0x7FC0).
+ *
+ * Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ * stream) of the current device; the library never synchronizes, allocates
+ * no memory and keeps no per-call state, so concurrent calls from several
+ * host threads are safe. All pointers must be device (or managed) memory of
+ * the current device. Argument errors are detected on the host before any
+ * launch and return a status; nothing is written in that case. Launch
+ * failures return MXQ_ERR_CUDA; faults during execution surface at the
+ * caller's next synchronization, as with any CUDA kernel.
+ */
+#ifndef MXQ_H
+#define MXQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MXQ_API __attribute__((visibility("default")))
+#else
+#define MXQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MXQ_AXS6 = 0,
+    MXQ_MXFP6_E2M3 = 1,
+    MXQ_MXFP6_E3M2 = 2,
+    MXQ_MXFP8_E4M3 = 3,
+    MXQ_MXFP4_E2M1 = 4
+} mxq_format;
+
+typedef enum { MXQ_F32 = 0, MXQ_BF16 = 1 } mxq_dtype;
+
+typedef enum {
+    MXQ_OK = 0,
+    MXQ_ERR_INVALID_ARG = 1, /* bad enum, null / host / other-device pointer          */
+    MXQ_ERR_SHAPE = 2,       /* rows < 0, cols <= 0, cols % 32 != 0, size overflow    */
+    MXQ_ERR_ALIGN = 3,       /* a pointer misses its alignment (see each call)        */
+    MXQ_ERR_UNSUPPORTED = 4, /* valid request this build does not implement           */
+    MXQ_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed                  */
+    MXQ_ERR_TIMEOUT = 6      /* a bounded device-side wait gave up (reserved)         */
+} mxq_status;
+
+/* A cudaStream_t, passed as an opaque pointer so this header needs no CUDA headers. */
+typedef void* mxq_stream;
+
+/*
+ * Quantize: values -> packed codes + scales.
+ *   src     [rows, cols] values of type `dtype`, 16-byte aligned.
+ *   codes   mxq_codes_bytes(fmt, rows, cols) bytes, 16-byte aligned.
+ *   scales  mxq_scales_bytes(fmt, rows, cols) bytes (2-byte aligned for AXS-6).
+ * rows == 0 is a valid no-op. src must not overlap codes or scales.
+ * Source: the block rule above ("AXS-6" block figure; "Sonar: Online MXFP6",
+ * Start a model; "EFQ-Softmax", stage table "Block scale").
+ */
+MXQ_API mxq_status mxq_quantize(mxq_format fmt, const void* src, mxq_dtype dtype, int64_t rows, int64_t cols,
+                        void* codes, void* scales, mxq_stream stream);
+
+/*
+ * Dequantize: codes + scales -> values of type `dtype`
+ *   value = decode(code) * 2^(scale byte - 127), rounded to nearest even into
+ *   `dtype` (exact except for bf16 results below 2^-126 and overflow).
+ *   codes   16-byte aligned; dst [rows, cols] 16-byte aligned; scales as above.
+ * dst must not overlap codes or scales.
+ */
+MXQ_API mxq_status mxq_dequantize(mxq_format fmt, const void* codes, const void* scales, int64_t rows, int64_t cols,
+                          void* dst, mxq_dtype dtype, mxq_stream stream);
+
+/*
+ * Fused fake-quantize: dst = dequantize(quantize(src)) in one pass, with no
+ * codes written to memory ("AXS-6", Quick Start Example: fused fake quantize
+ * with block_size=32, no intermediate allocation). dst has src's type and
+ * shape; dst == src (in place) is allowed, any other overlap is not. Both
+ * 16-byte aligned.
+ */
+MXQ_API mxq_status mxq_fake_quantize(mxq_format fmt, const void* src, mxq_dtype dtype, int64_t rows, int64_t cols,
+                             void* dst, mxq_stream stream);
+
+/*
+ * Exp-then-quantize softmax probability stage ("EFQ-Softmax" explainer,
+ * Jargon: shifted scores, exp-then-quantize; stage table: probability
+ * generation, block scale). For every row r:
+ *   m   = max_j scores[r, j]            (NaN if the row holds a NaN)
+ *   p_j = expf_mxq(scores[r, j] - m)     (fp32 subtraction, then the library's
+ *                                         own deterministic fp32 exponential:
+ *                                         Cody-Waite reduction by ln 2 split in
+ *                                         two constants, degree-7 Taylor
+ *                                         polynomial in fused multiply-adds)
+ *   then p is block-quantized exactly like mxq_quantize with dtype MXQ_F32.
+ * p is never written to memory. Supported formats: all five (MXFP4 E2M1 is
+ * the one the stage feeds). scores 16-byte aligned, cols <= 131072
+ * (MXQ_ERR_UNSUPPORTED above that).
+ */
+MXQ_API mxq_status mxq_exp_quantize(mxq_format fmt, const float* scores, int64_t rows, int64_t cols,
+                            void* codes, void* scales, mxq_stream stream);
+
+/*
+ * Grouped quantize: n independent tensors of one format and one value type
+ * converted by a single launch (a decoder layer's seven weight matrices in the
+ * online layer-by-layer conversion of "Sonar: Online MXFP6", Start a model).
+ * Each descriptor obeys the rules of mxq_quantize. 1 <= n <= MXQ_MAX_GROUP.
+ * The descriptor array is read on the host during the call only.
+ */
+#define MXQ_MAX_GROUP 64
+typedef struct {
+    const void* src;
+    void* codes;
+    void* scales;
+    int64_t rows;
+    int64_t cols;
+} mxq_tensor;
+
+MXQ_API mxq_status mxq_quantize_grouped(mxq_format fmt, mxq_dtype dtype, const mxq_tensor* tensors, int n,
+                                mxq_stream stream);
+
+/* Bytes of the packed code array: rows * cols/32 * payload (0 on bad input). */
+MXQ_API size_t mxq_codes_bytes(mxq_format fmt, int64_t rows, int64_t cols);
+/* Bytes of the scale array: rows * cols/32 (x2 for AXS-6 headers; 0 on bad input). */
+MXQ_API size_t mxq_scales_bytes(mxq_format fmt, int64_t rows, int64_t cols);
+/* Information bits per block: 8 scale bits + 32 * element bits, plus the
+ * 2-bit config field for AXS-6 -> 202, 200, 200, 264, 136; -1 on bad input. */
+MXQ_API int mxq_block_bits(mxq_format fmt);
+/* Static, human-readable description of a status code. */
+MXQ_API const char* mxq_status_string(mxq_status status);
+/* Library version, "major.minor.patch". */
+MXQ_API const char* mxq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXQ_H */

@@ -1,0 +1,105 @@
+"""The C ABI library loads and exports every symbol include/mxq.h declares;
+host-only behaviour (size queries, statuses returned before any CUDA call).
+No kernel runs here."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import oracle
+from block_scaled_microscaling_b200 import build as mxq_build
+from block_scaled_microscaling_b200 import mxq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mxq.h")
+FMTS = ["axs6", "mxfp6_e2m3", "mxfp6_e3m2", "mxfp8", "mxfp4"]
+
+
+@pytest.fixture(scope="module")
+def L():
+    mxq_build.build()
+    return mxq.lib()
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return re.findall(r"MXQ_API\s+[\w\s\*]+?\b(mxq_\w+)\s*\(", src)
+
+
+def test_exports_every_declared_symbol(L):
+    syms = declared_symbols()
+    assert len(syms) == 10
+    out = subprocess.run(["nm", "-D", "--defined-only", mxq.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT\s+(mxq_\w+)", out))
+    for s in syms:
+        assert s in exported, s
+        assert hasattr(L, s)
+    assert set(mxq.EXPORTS) == set(syms)
+
+
+def test_enum_values_match_header():
+    src = open(HEADER).read()
+    for name, v in [("MXQ_AXS6", 0), ("MXQ_MXFP6_E2M3", 1), ("MXQ_MXFP6_E3M2", 2), ("MXQ_MXFP8_E4M3", 3),
+                    ("MXQ_MXFP4_E2M1", 4), ("MXQ_F32", 0), ("MXQ_BF16", 1), ("MXQ_OK", 0),
+                    ("MXQ_ERR_INVALID_ARG", 1), ("MXQ_ERR_SHAPE", 2), ("MXQ_ERR_ALIGN", 3),
+                    ("MXQ_ERR_UNSUPPORTED", 4), ("MXQ_ERR_CUDA", 5), ("MXQ_ERR_TIMEOUT", 6)]:
+        assert re.search(rf"\b{name}\s*=\s*{v}\b", src), name
+    assert list(mxq.FORMATS.values()) == [0, 1, 2, 3, 4]
+    assert re.search(r"#define MXQ_MAX_GROUP\s+(\d+)", src).group(1) == str(mxq.MAX_GROUP)
+
+
+def test_block_bits_match_page_facts(L):
+    # 8 scale bits + 32 elements, plus AXS-6's 2-bit config ("AXS-6" block figure)
+    assert [mxq.mxq_block_bits(i) for i in range(5)] == [202, 200, 200, 264, 136]
+    assert round(mxq.mxq_block_bits(0) / 32, 2) == 6.31
+    assert mxq.mxq_block_bits(7) == -1
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_size_queries_match_oracle(L, fmt):
+    for rows, cols in [(1, 32), (3, 96), (4096, 4096), (16384, 8192), (0, 64)]:
+        f = mxq.FORMATS[fmt]
+        assert mxq.mxq_codes_bytes(f, rows, cols) == oracle.lib().orc_codes_bytes(oracle.FORMATS[fmt], rows, cols)
+        assert mxq.mxq_scales_bytes(f, rows, cols) == oracle.lib().orc_scales_bytes(oracle.FORMATS[fmt], rows, cols)
+    assert mxq.mxq_codes_bytes(mxq.FORMATS[fmt], 2, 33) == 0
+    assert mxq.mxq_scales_bytes(mxq.FORMATS[fmt], -1, 32) == 0
+
+
+def test_statuses_before_any_cuda_call(L):
+    q = mxq.mxq_quantize
+    assert q(9, None, 0, 1, 32, None, None, None) == 1          # bad format
+    assert q(1, None, 5, 1, 32, None, None, None) == 1          # bad dtype
+    assert q(1, None, 0, 1, 33, None, None, None) == 2          # cols % 32
+    assert q(1, None, 0, -1, 32, None, None, None) == 2         # rows < 0
+    assert q(1, None, 0, 1, 0, None, None, None) == 2           # cols == 0
+    assert q(1, None, 0, 1 << 40, 1 << 20, None, None, None) == 2  # size overflow
+    assert q(1, None, 0, 0, 32, None, None, None) == 0          # empty: no-op
+    assert q(1, None, 0, 1, 32, None, None, None) == 1          # null pointer
+    assert mxq.mxq_dequantize(1, None, None, 0, 64, None, 1, None) == 0
+    assert mxq.mxq_dequantize(1, None, None, 2, 64, None, 3, None) == 1
+    assert mxq.mxq_fake_quantize(0, None, 0, 0, 64, None, None) == 0
+    assert mxq.mxq_fake_quantize(0, None, 0, 1, 48, None, None) == 2
+    assert mxq.mxq_exp_quantize(4, None, 0, 64, None, None, None) == 0
+    assert mxq.mxq_exp_quantize(4, None, 2, 40, None, None, None) == 2
+    assert mxq.mxq_quantize_grouped(1, 1, [], None) == 1
+    assert mxq.mxq_quantize_grouped(1, 1, [(0, 0, 0, 0, 64)], None) == 0
+    assert mxq.mxq_quantize_grouped(1, 1, [(0, 0, 0, 0, 64)] * 65, None) == 1
+    for s in range(7):
+        assert mxq.mxq_status_string(s)
+    assert mxq.mxq_status_string(99) == "unknown status"
+    assert mxq.mxq_version().count(".") == 2
+
+
+def test_block_size_other_than_32_is_rejected():
+    with pytest.raises(mxq.MXQError) as e:
+        mxq.fake_quantize(None, "axs6", block_size=16)
+    assert e.value.status == 4
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(mxq, "LIB_PATH", str(tmp_path / "libmxq.so"))
+    monkeypatch.setattr(mxq, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        mxq.lib()
