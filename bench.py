@@ -173,6 +173,23 @@ def run_reference(args, rank, world):
     return 0
 
 
+# ---- multi-rank host logic (replicas; no data-path collective) ---------------------------
+
+def max_over_ranks(value, dist, device):
+    """The largest `value` over all ranks (timing only); identity on one process."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(world, bytes_per_step, steps, ms_total_max):
+    """Whole-job throughput: every rank moved bytes_per_step * steps; time = slowest rank."""
+    return world * bytes_per_step * steps / (ms_total_max * 1e-3) / 1e9
+
+
 # ---- the GPU arm --------------------------------------------------------------------------
 
 def make_sets(torch, mxq, w_dev, nsets):
@@ -364,8 +381,57 @@ def workloads_breakdown(torch, mxq, hbm):
     return out
 
 
+PROFILE_CASES = ["q_e2m3_weight", "dq_e2m3_weight", "q_mxfp8_act", "dq_mxfp8_act", "q_axs6_layer",
+                 "q_e2m3_layer", "fq_axs6_grad", "exp_mxfp4_scores"]
+
+
+def profile_case(name, reps):
+    """Run one kernel `reps` times on its workload (for ncu captures); prints one line."""
+    import torch
+    from block_scaled_microscaling_b200 import mxq
+    dev = torch.device("cuda")
+    gen = torch.Generator(device=dev).manual_seed(0)
+    if name in ("q_e2m3_weight", "dq_e2m3_weight"):
+        w_host, _ = synthetic.weight_with_outliers(seed=1)
+        x = torch.from_numpy(w_host.view(np.int16)).view(torch.bfloat16).cuda()
+        c, s = mxq.quantize(x, "mxfp6_e2m3")
+        y = torch.empty_like(x)
+        fn = (lambda: mxq.quantize(x, "mxfp6_e2m3", codes=c, scales=s)) if name[0] == "q" else \
+            (lambda: mxq.dequantize(c, s, "mxfp6_e2m3", x.shape, out=y))
+    elif name in ("q_mxfp8_act", "dq_mxfp8_act"):
+        x = (torch.randn(16384, 8192, device=dev, generator=gen) * 0.5).to(torch.bfloat16)
+        c, s = mxq.quantize(x, "mxfp8")
+        y = torch.empty_like(x)
+        fn = (lambda: mxq.quantize(x, "mxfp8", codes=c, scales=s)) if name[0] == "q" else \
+            (lambda: mxq.dequantize(c, s, "mxfp8", x.shape, out=y))
+    elif name in ("q_axs6_layer", "q_e2m3_layer"):
+        fmt = "axs6" if "axs6" in name else "mxfp6_e2m3"
+        ws = [(torch.randn(r, c_, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+              for _, r, c_ in synthetic.DECODER_LAYER]
+        outs = mxq.quantize_grouped(ws, fmt)
+        fn = lambda: mxq.quantize_grouped(ws, fmt, outs=outs)
+    elif name == "fq_axs6_grad":
+        g = torch.randn(16384, 8192, device=dev, generator=gen) * 1e-3
+        o = torch.empty_like(g)
+        fn = lambda: mxq.fake_quantize(g, "axs6", out=o)
+    elif name == "exp_mxfp4_scores":
+        sc = torch.randn(4096, 32768, device=dev, generator=gen) * 3
+        c, s = mxq.exp_quantize(sc, "mxfp4")
+        fn = lambda: mxq.exp_quantize(sc, "mxfp4", codes=c, scales=s)
+    else:
+        raise SystemExit(f"unknown profile case {name}; one of {PROFILE_CASES}")
+    for _ in range(reps):
+        fn()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": name, "reps": reps}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--profile-case", choices=PROFILE_CASES, default=None,
+                    help="run one kernel a few times on its workload and exit (for ncu captures)")
+    ap.add_argument("--profile-reps", type=int, default=3)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=16)
@@ -382,6 +448,8 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.profile_case:
+        return profile_case(args.profile_case, args.profile_reps)
 
     import torch
     import torch.distributed as dist
@@ -409,6 +477,7 @@ def main():
     gw.replay()
     torch.cuda.synchronize()
     gt, events, names = capture(torch, mxq, sets, args.warmup, args.steps, True)
+    gp, _, _ = capture(torch, mxq, sets, args.warmup, args.steps, False)
     torch.cuda.synchronize()
 
     start = torch.cuda.Event(enable_timing=True)
@@ -424,18 +493,24 @@ def main():
     if world > 1:
         dist.barrier()
     ms_total = start.elapsed_time(end)
+    # the same K steps without the per-launch timing events (their cost, for the record)
+    gp.replay()
+    torch.cuda.synchronize()
+    start.record()
+    gp.replay()
+    end.record()
+    torch.cuda.synchronize()
+    ms_plain = start.elapsed_time(end)
+    del gp
     per_op = {nm: [] for nm in names}
     for ev in events:
         for j, nm in enumerate(names):
             per_op[nm].append(ev[j].elapsed_time(ev[j + 1]))
-    if world > 1:
-        t = torch.tensor([ms_total], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, dist if world > 1 else None, "cuda")
     del gt, gw
 
     ms_step = ms_total / args.steps
-    value = world * step_bytes * args.steps / (ms_total * 1e-3) / 1e9
+    value = job_gbs(world, step_bytes, args.steps, ms_total)
     op_ms = {nm: statistics.mean(v) for nm, v in per_op.items()}
     dominant = max(op_ms, key=op_ms.get)
     ach = op_bytes / (op_ms[dominant] * 1e-3) / 1e9
@@ -447,7 +522,8 @@ def main():
         "config": {"workload": WORKLOAD, "elements": n, "bytes_per_step": step_bytes,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "8 rotating buffer sets (~1 GB): each launch reads data last touched >= 4 steps earlier",
-                   "timing": "one CUDA graph of K steps, CUDA events on the launching stream"},
+                   "timing": "one CUDA graph of K steps, CUDA events on the launching stream",
+                   "ms_per_step_without_inner_events": round(ms_plain / args.steps, 5)},
         "frac_hbm": round(value / world / hbm, 4),
         "per_op": {nm: {"ms": round(v, 5), "GB/s": round(op_bytes / (v * 1e-3) / 1e9, 1),
                         "frac_hbm": round(op_bytes / (v * 1e-3) / 1e9 / hbm, 4)} for nm, v in op_ms.items()},
