@@ -8,10 +8,11 @@ reverse) / device time, GB/s, and the fraction of the measured HBM copy peak.
 
 Timing: 8 rotating buffer sets (~1 GB) so that every launch reads data last
 touched >= 4 steps (>700 MB of traffic) earlier, i.e. from HBM, not L2; the
-timed K steps are one CUDA graph (4 kernel nodes per step, a timing event
-between consecutive launches), replayed once between CUDA events on the
-launching stream; clocks and throttle reasons are sampled through NVML while
-it runs. e2e: the same step through the public Python API from pinned host
+timed K steps are one CUDA graph (4 kernel nodes per step, nothing between
+them) replayed once between CUDA events on the launching stream; clocks and
+throttle reasons are sampled through NVML while it runs. Per-kernel average
+durations (the roofline's `achieved`) come from one more graph per kernel: K
+back-to-back launches of it on the same rotation, timed as a whole. e2e: the same step through the public Python API from pinned host
 memory, host->device copy of the weight and device->host copy of every
 output inside the timed region. cpu_baseline: the CPU oracle on a bounded
 row sample of the same workload.
@@ -218,30 +219,31 @@ def step_ops(mxq, sets, k):
     ]
 
 
-def capture(torch, mxq, sets, k0, nsteps, with_events):
-    """One CUDA graph holding nsteps steps; events[k][j] brackets launch j of step k."""
+def graph_of(torch, fns):
+    """One CUDA graph that launches every callable of `fns` in order on one stream."""
     g = torch.cuda.CUDAGraph()
-    events = []
     stream = torch.cuda.Stream()
     stream.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(stream):
         with torch.cuda.graph(g, stream=stream):
-            for k in range(k0, k0 + nsteps):
-                ops = step_ops(mxq, sets, k)
-                ev = []
-                for name, fn in ops:
-                    if with_events:
-                        e = torch.cuda.Event(enable_timing=True, external=True)
-                        e.record()
-                        ev.append(e)
-                    fn()
-                if with_events:
-                    e = torch.cuda.Event(enable_timing=True, external=True)
-                    e.record()
-                    ev.append(e)
-                events.append(ev)
+            for fn in fns:
+                fn()
     torch.cuda.current_stream().wait_stream(stream)
-    return g, events, [n for n, _ in step_ops(mxq, sets, 0)]
+    return g
+
+
+def time_graph(torch, g, replays=1):
+    """Device time (ms) of `replays` back-to-back replays, CUDA events on the launching stream."""
+    g.replay()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(replays):
+        g.replay()
+    end.record()
+    torch.cuda.synchronize()
+    return start.elapsed_time(end)
 
 
 def e2e_measure(torch, mxq, w_host, steps):
@@ -279,34 +281,13 @@ def e2e_measure(torch, mxq, w_host, steps):
 
 
 def time_launches(torch, fns, reps):
-    """Mean device time of each launch in `fns`, repeated `reps` times round-robin,
-    one CUDA graph with an event between consecutive launches."""
-    g = torch.cuda.CUDAGraph()
-    stream = torch.cuda.Stream()
-    stream.wait_stream(torch.cuda.current_stream())
-    evs = []
-    with torch.cuda.stream(stream):
-        with torch.cuda.graph(g, stream=stream):
-            for r in range(reps):
-                for fn in fns:
-                    e = torch.cuda.Event(enable_timing=True, external=True)
-                    e.record()
-                    evs.append(e)
-                    fn()
-            e = torch.cuda.Event(enable_timing=True, external=True)
-            e.record()
-            evs.append(e)
-    torch.cuda.current_stream().wait_stream(stream)
-    g.replay()
-    torch.cuda.synchronize()
-    g.replay()
-    torch.cuda.synchronize()
-    n = len(fns)
-    ts = [[] for _ in range(n)]
-    for i in range(len(evs) - 1):
-        ts[i % n].append(evs[i].elapsed_time(evs[i + 1]))
-    del g
-    return [statistics.mean(t) for t in ts]
+    """Mean device time of each callable: a graph of `reps` back-to-back launches of it, timed as a whole."""
+    out = []
+    for fn in fns:
+        g = graph_of(torch, [fn] * reps)
+        out.append(time_graph(torch, g) / reps)
+        del g
+    return out
 
 
 def workloads_breakdown(torch, mxq, hbm):
@@ -342,8 +323,10 @@ def workloads_breakdown(torch, mxq, hbm):
     for fmt in ("mxfp6_e2m3", "axs6"):
         outs = [mxq.quantize_grouped(ws, fmt) for ws in layers]
         fns = [lambda ws=ws, o=o: mxq.quantize_grouped(ws, fmt, outs=o) for ws, o in zip(layers, outs)]
-        ts = time_launches(torch, fns, 2)
-        rec(f"c3_stack_{fmt}_quantize_bf16", nbytes_q(fmt, n3, 2), n3, sum(ts))
+        g = graph_of(torch, fns * 2)
+        ms = time_graph(torch, g) / 2
+        del g
+        rec(f"c3_stack_{fmt}_quantize_bf16", nbytes_q(fmt, n3, 2), n3, ms)
         del outs
     del layers
     torch.cuda.empty_cache()
@@ -468,18 +451,19 @@ def main():
     op_bytes = nbytes_q("mxfp6_e2m3", n, 2)  # same for all four launches
     step_bytes = 4 * op_bytes
 
-    # warm-up: eager, then a captured graph of W steps
+    # warm-up: eager W steps, then the same W steps as a graph
     for k in range(args.warmup):
         for _, fn in step_ops(mxq, sets, k):
             fn()
     torch.cuda.synchronize()
-    gw, _, _ = capture(torch, mxq, sets, 0, args.warmup, False)
+    names = [nm for nm, _ in step_ops(mxq, sets, 0)]
+    gw = graph_of(torch, [fn for k in range(args.warmup) for _, fn in step_ops(mxq, sets, k)])
     gw.replay()
     torch.cuda.synchronize()
-    gt, events, names = capture(torch, mxq, sets, args.warmup, args.steps, True)
-    gp, _, _ = capture(torch, mxq, sets, args.warmup, args.steps, False)
+    # timed region: K steps (4 launches each) as one graph, no events between launches
+    gt = graph_of(torch, [fn for k in range(args.warmup, args.warmup + args.steps)
+                          for _, fn in step_ops(mxq, sets, k)])
     torch.cuda.synchronize()
-
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -493,25 +477,17 @@ def main():
     if world > 1:
         dist.barrier()
     ms_total = start.elapsed_time(end)
-    # the same K steps without the per-launch timing events (their cost, for the record)
-    gp.replay()
-    torch.cuda.synchronize()
-    start.record()
-    gp.replay()
-    end.record()
-    torch.cuda.synchronize()
-    ms_plain = start.elapsed_time(end)
-    del gp
-    per_op = {nm: [] for nm in names}
-    for ev in events:
-        for j, nm in enumerate(names):
-            per_op[nm].append(ev[j].elapsed_time(ev[j + 1]))
-    ms_total = max_over_ranks(ms_total, dist if world > 1 else None, "cuda")
     del gt, gw
+    # per-kernel average duration: K back-to-back launches of one op (same rotation, cold data)
+    op_ms = {}
+    for j, nm in enumerate(names):
+        g = graph_of(torch, [step_ops(mxq, sets, k)[j][1] for k in range(args.steps)])
+        op_ms[nm] = time_graph(torch, g) / args.steps
+        del g
+    ms_total = max_over_ranks(ms_total, dist if world > 1 else None, "cuda")
 
     ms_step = ms_total / args.steps
     value = job_gbs(world, step_bytes, args.steps, ms_total)
-    op_ms = {nm: statistics.mean(v) for nm, v in per_op.items()}
     dominant = max(op_ms, key=op_ms.get)
     ach = op_bytes / (op_ms[dominant] * 1e-3) / 1e9
 
@@ -522,8 +498,8 @@ def main():
         "config": {"workload": WORKLOAD, "elements": n, "bytes_per_step": step_bytes,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "8 rotating buffer sets (~1 GB): each launch reads data last touched >= 4 steps earlier",
-                   "timing": "one CUDA graph of K steps, CUDA events on the launching stream",
-                   "ms_per_step_without_inner_events": round(ms_plain / args.steps, 5)},
+                   "timing": "one CUDA graph of K steps replayed between CUDA events on the launching stream; "
+                             "per-kernel: a graph of K launches of that kernel alone"},
         "frac_hbm": round(value / world / hbm, 4),
         "per_op": {nm: {"ms": round(v, 5), "GB/s": round(op_bytes / (v * 1e-3) / 1e9, 1),
                         "frac_hbm": round(op_bytes / (v * 1e-3) / 1e9 / hbm, 4)} for nm, v in op_ms.items()},

@@ -1,0 +1,225 @@
+// mxq_block.cuh -- one block of 32 values: load, maximum, encode to a packed
+// payload, decode back (sm_100a). Shared by the codec and softmax kernels.
+//
+// Block rule ("AXS-6: Adaptive eXponent Sharing", block figure; "Sonar: Online
+// MXFP6", Start a model; "EFQ-Softmax" stage table): one E8M0 scale from the
+// block's absolute maximum, values rounded to nearest even with saturation,
+// codes packed LSB-first (value j at bits [W*j, W*j+W) of the payload).
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "mxq_device.cuh"
+
+namespace mxq {
+
+template <typename T> struct Blk { static constexpr int NW = 32 * (int)sizeof(T) / 4; };  // words per block
+
+// ---- values in ----------------------------------------------------------------------
+
+template <typename T>
+__device__ __forceinline__ void load_block(const void* base, long long b, uint32_t* w, bool a32) {
+    const char* p = reinterpret_cast<const char*>(base) + b * 32 * (long long)sizeof(T);
+#pragma unroll
+    for (int i = 0; i < Blk<T>::NW / 8; ++i) ld32(p + 32 * i, w + 8 * i, a32);
+}
+
+// fp32 bit pattern of max |x| over the block (NaN -> a pattern above 0x7F800000)
+template <typename T> __device__ __forceinline__ uint32_t block_amax(const uint32_t* w);
+template <> __device__ __forceinline__ uint32_t block_amax<__nv_bfloat16>(const uint32_t* w) {
+    uint32_t m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = absmax_bf16x2(w[2 * i], w[2 * i + 1]);
+#pragma unroll
+    for (int s = 4; s > 0; s >>= 1)
+#pragma unroll
+        for (int i = 0; i < s; ++i) m[i] = absmax_bf16x2(m[i], m[i + s]);
+    return max((m[0] & 0x7FFFu) << 16, m[0] & 0x7FFF0000u);
+}
+template <> __device__ __forceinline__ uint32_t block_amax<float>(const uint32_t* w) {
+    float m[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m[i] = absmax_f32(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1]));
+#pragma unroll
+    for (int s = 8; s > 0; s >>= 1)
+#pragma unroll
+        for (int i = 0; i < s; ++i) m[i] = absmax_f32(m[i], m[i + s]);
+    return __float_as_uint(m[0]) & 0x7FFFFFFFu;
+}
+
+// values 2i, 2i+1 of the block as a packed fp32 pair
+template <typename T> __device__ __forceinline__ unsigned long long pair(const uint32_t* w, int i);
+template <> __device__ __forceinline__ unsigned long long pair<__nv_bfloat16>(const uint32_t* w, int i) {
+    return pk(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+}
+template <> __device__ __forceinline__ unsigned long long pair<float>(const uint32_t* w, int i) {
+    return pk(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1]));
+}
+// ---- codes of one block ---------------------------------------------------------------
+//
+// Each format produces, for pair i (values 2i, 2i+1), a small integer h_i
+// holding code(2i) in its low W bits and code(2i+1) above it, then the pairs
+// are packed LSB-first into the payload words.
+
+// 6-bit: two codes one per byte -> 12-bit field c0 | c1 << 6
+__device__ __forceinline__ uint32_t squeeze6(uint32_t h) { return h - 192u * (h >> 8); }
+
+template <int F, typename T>
+__device__ __forceinline__ uint32_t code_pair(const uint32_t* w, int i, float inv) {
+    float a, b;
+    upk(f2mul(pair<T>(w, i), dup2(inv)), a, b);
+    if constexpr (F == F_AXS6) {
+        // sign | min(rne(16|y|), 31), rne by a 1.5*2^23 add; the x16 is exact
+        uint32_t ma = __float_as_uint(fabsf(a) * 16.0f + 12582912.0f) - 0x4B400000u;
+        uint32_t mb = __float_as_uint(fabsf(b) * 16.0f + 12582912.0f) - 0x4B400000u;
+        ma = min(ma, 31u) | ((__float_as_uint(a) >> 26) & 0x20u);
+        mb = min(mb, 31u) | ((__float_as_uint(b) >> 26) & 0x20u);
+        return ma | (mb << 6);
+    } else if constexpr (Fmt<F>::W == 6) {
+        return squeeze6(cvt2<F>(a, b));
+    } else {
+        return cvt2<F>(a, b);  // E4M3: 16 bits, E2M1: 8 bits
+    }
+}
+
+// payload words of a block (P/4 of them: 6-bit 6, E4M3 8, E2M1 4)
+template <int F, typename T>
+__device__ __forceinline__ void encode_block(const uint32_t* w, uint32_t byte, uint32_t* out) {
+    const float inv = inv_scale(byte);
+    const uint32_t keep = byte == 0xFFu ? 0u : 0xFFFFFFFFu;
+    if constexpr (Fmt<F>::W == 6) {
+        uint32_t z[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) z[j] = (code_pair<F, T>(w, 2 * j, inv) | (code_pair<F, T>(w, 2 * j + 1, inv) << 12)) & keep;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const uint32_t* q = z + 4 * k;
+            out[3 * k + 0] = q[0] | (q[1] << 24);
+            out[3 * k + 1] = (q[1] >> 8) | (q[2] << 16);
+            out[3 * k + 2] = (q[2] >> 16) | (q[3] << 8);
+        }
+    } else if constexpr (Fmt<F>::W == 8) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) out[j] = (code_pair<F, T>(w, 2 * j, inv) | (code_pair<F, T>(w, 2 * j + 1, inv) << 16)) & keep;
+    } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            out[j] = (code_pair<F, T>(w, 4 * j, inv) | (code_pair<F, T>(w, 4 * j + 1, inv) << 8) |
+                      (code_pair<F, T>(w, 4 * j + 2, inv) << 16) | (code_pair<F, T>(w, 4 * j + 3, inv) << 24)) & keep;
+    }
+}
+
+template <int F>
+__device__ __forceinline__ void store_payload(void* codes, long long b, const uint32_t* out, bool a32) {
+    char* p = reinterpret_cast<char*>(codes) + b * payload<F>();
+    if constexpr (Fmt<F>::W == 6) {  // 24 bytes at a multiple of 8
+        uint2* q = reinterpret_cast<uint2*>(p);
+        q[0] = make_uint2(out[0], out[1]);
+        q[1] = make_uint2(out[2], out[3]);
+        q[2] = make_uint2(out[4], out[5]);
+    } else if constexpr (Fmt<F>::W == 8) {
+        st32(p, out, a32);
+    } else {
+        st_stream_v4(p, make_uint4(out[0], out[1], out[2], out[3]));
+    }
+}
+template <int F>
+__device__ __forceinline__ void load_payload(const void* codes, long long b, uint32_t* out, bool a32) {
+    const char* p = reinterpret_cast<const char*>(codes) + b * payload<F>();
+    if constexpr (Fmt<F>::W == 6) {  // 3 x 8 bytes, through L1 so the partial sectors are fetched once
+        const uint2* q = reinterpret_cast<const uint2*>(p);
+        uint2 a = __ldg(q), c = __ldg(q + 1), d = __ldg(q + 2);
+        out[0] = a.x; out[1] = a.y; out[2] = c.x; out[3] = c.y; out[4] = d.x; out[5] = d.y;
+    } else if constexpr (Fmt<F>::W == 8) {
+        ld32(p, out, a32);
+    } else {
+        uint4 v = ld_stream_v4(p);
+        out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+    }
+}
+
+template <int F>
+__device__ __forceinline__ void store_scale(void* scales, long long b, uint32_t byte) {
+    if constexpr (Fmt<F>::FIXED) reinterpret_cast<uint16_t*>(scales)[b] = (uint16_t)byte;  // config = 0
+    else reinterpret_cast<uint8_t*>(scales)[b] = (uint8_t)byte;
+}
+template <int F>
+__device__ __forceinline__ uint32_t load_scale(const void* scales, long long b) {
+    if constexpr (Fmt<F>::FIXED) return __ldg(reinterpret_cast<const uint16_t*>(scales) + b) & 0xFFu;
+    else return __ldg(reinterpret_cast<const uint8_t*>(scales) + b);
+}
+
+// ---- decoding ---------------------------------------------------------------------------
+
+// code k (0..31) of a payload as the fp32 pattern of decode(code) * 2^-(127-BIAS)
+// (AXS-6: * 2^-126): magnitude onto the exponent/mantissa fields, sign to bit 31.
+template <int F>
+__device__ __forceinline__ uint32_t payload_bits(const uint32_t* pw, int k) {
+    constexpr int W = Fmt<F>::W;
+    constexpr int SH = Fmt<F>::FIXED ? 19 : 23 - Fmt<F>::M;
+    const int bit = W * k;
+    uint32_t c;
+    if constexpr (W == 6) {
+        const int lo = bit & 31;  // fields may straddle two words
+        c = (lo <= 26) ? (pw[bit >> 5] >> lo) : ((pw[bit >> 5] >> lo) | (pw[(bit >> 5) + 1] << (32 - lo)));
+    } else {
+        c = pw[bit >> 5] >> (bit & 31);
+    }
+    return ((c & ((1u << (W - 1)) - 1u)) << SH) | ((c << (32 - W)) & 0x80000000u);
+}
+
+// output: 32 values of the block as output words (bf16 pairs or fp32)
+template <int F, typename T>
+__device__ __forceinline__ void decode_block(const uint32_t* pw, uint32_t byte, uint32_t* o) {
+    const float s = fwd_scale(byte);
+    const unsigned long long D = dup2(decode_unit<F>()), S = dup2(s);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        float a, b;
+        upk(f2mul(f2mul(pk(__uint_as_float(payload_bits<F>(pw, 2 * i)), __uint_as_float(payload_bits<F>(pw, 2 * i + 1))), D), S),
+            a, b);
+        if constexpr (sizeof(T) == 4) {
+            o[2 * i] = __float_as_uint(a);
+            o[2 * i + 1] = __float_as_uint(b);
+        } else {
+            o[i] = bf16x2(a, b);
+        }
+    }
+    // E4M3's NaN magnitude (0x7F) and NaN blocks: canonical quiet NaN
+    if constexpr (F == F_E4M3) {
+        uint32_t nan_bytes = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) nan_bytes |= ((pw[j] & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u;
+        if (nan_bytes) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                if (((pw[k >> 2] >> (8 * (k & 3))) & 0x7Fu) == 0x7Fu) {
+                    if constexpr (sizeof(T) == 4) o[k] = 0x7FC00000u;
+                    else o[k >> 1] = (k & 1) ? ((o[k >> 1] & 0x0000FFFFu) | 0x7FC00000u) : ((o[k >> 1] & 0xFFFF0000u) | 0x7FC0u);
+                }
+            }
+        }
+    }
+    if (byte == 0xFFu) {
+#pragma unroll
+        for (int i = 0; i < Blk<T>::NW; ++i) o[i] = sizeof(T) == 4 ? 0x7FC00000u : 0x7FC07FC0u;
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ void store_block(void* dst, long long b, const uint32_t* o, bool a32) {
+    char* p = reinterpret_cast<char*>(dst) + b * 32 * (long long)sizeof(T);
+#pragma unroll
+    for (int i = 0; i < Blk<T>::NW / 8; ++i) st32(p + 32 * i, o + 8 * i, a32);
+}
+
+// fake-quantize of one block: codes computed and decoded in registers
+template <int F, typename T>
+__device__ __forceinline__ void fake_block(const uint32_t* w, uint32_t byte, uint32_t* o) {
+    uint32_t pw[8];
+    encode_block<F, T>(w, byte, pw);
+    decode_block<F, T>(pw, byte, o);
+}
+
+}  // namespace mxq

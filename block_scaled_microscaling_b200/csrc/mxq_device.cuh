@@ -44,6 +44,38 @@ __device__ __forceinline__ void st_stream_v4(void* p, uint4 v) {
     asm volatile("st.global.L1::no_allocate.v4.u32 [%0], {%1,%2,%3,%4};"
                  :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
+// 32 bytes = one DRAM sector per lane (sm_100 256-bit accesses); p 32-byte aligned
+__device__ __forceinline__ void ld_v8(const void* p, uint32_t* r) {
+    asm volatile("ld.global.nc.L1::no_allocate.L2::evict_first.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "l"(p));
+}
+__device__ __forceinline__ void st_v8(void* p, const uint32_t* r) {
+    asm volatile("st.global.L1::no_allocate.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 :: "l"(p), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+// 16-byte halves through L1 (the second half of a sector then hits L1); p 16-byte aligned
+__device__ __forceinline__ void ld_2v4(const void* p, uint32_t* r) {
+    uint4 a, b;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w) : "l"(p));
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w) : "l"(reinterpret_cast<const char*>(p) + 16));
+    r[0] = a.x; r[1] = a.y; r[2] = a.z; r[3] = a.w; r[4] = b.x; r[5] = b.y; r[6] = b.z; r[7] = b.w;
+}
+__device__ __forceinline__ void st_2v4(void* p, const uint32_t* r) {
+    st_stream_v4(p, make_uint4(r[0], r[1], r[2], r[3]));
+    st_stream_v4(reinterpret_cast<char*>(p) + 16, make_uint4(r[4], r[5], r[6], r[7]));
+}
+// 32 bytes at p: one 256-bit access when a32, else two 128-bit ones
+__device__ __forceinline__ void ld32(const void* p, uint32_t* r, bool a32) {
+    if (a32) ld_v8(p, r);
+    else ld_2v4(p, r);
+}
+__device__ __forceinline__ void st32(void* p, const uint32_t* r, bool a32) {
+    if (a32) st_v8(p, r);
+    else st_2v4(p, r);
+}
 
 // ---------------------------------------------------------------------------
 // packed fp32 pair arithmetic (one instruction for two IEEE round-to-nearest ops)
@@ -60,6 +92,51 @@ __device__ __forceinline__ void mul2(float& a, float& b, float s) {
     unsigned long long r;
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(pk(a, b)), "l"(pk(s, s)));
     upk(r, a, b);
+}
+// packed pair ops on 64-bit {lo, hi} values
+__device__ __forceinline__ unsigned long long f2mul(unsigned long long a, unsigned long long b) {
+    unsigned long long r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ unsigned long long f2add(unsigned long long a, unsigned long long b) {
+    unsigned long long r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ unsigned long long f2sub(unsigned long long a, unsigned long long b) {
+    unsigned long long r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ unsigned long long f2fma(unsigned long long a, unsigned long long b, unsigned long long c) {
+    unsigned long long r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ unsigned long long dup2(float s) { return pk(s, s); }
+
+// NaN-propagating maxima (a NaN operand gives NaN); |a|,|b| variants for amax
+__device__ __forceinline__ float max_nan(float a, float b) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float max3_nan(float a, float b, float c) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+// max(|a|, |b|) of two bf16 pairs, lane-wise; NaN -> NaN (sign bits of the result are not meaningful)
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ __forceinline__ float absmax_f32(float a, float b) {
+    float r;
+    asm("max.NaN.xorsign.abs.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
 }
 
 // ---------------------------------------------------------------------------

@@ -5,19 +5,19 @@
 // conventional path exponentiates the row-max-shifted scores in higher
 // precision, materializes the probability block and quantizes it to E2M1 with
 // an exponent-only scale from each 32-key block's maximum. Here the block is
-// never materialized: scores are read once, probabilities live in registers.
+// never materialized: scores are read once and probabilities live in registers.
 //
-// One thread-block cluster per row. The row is split into C <= 8 contiguous
-// runs of whole 32-key blocks, one per CTA; each thread keeps up to R = 4
-// 16-byte chunks (16 scores) in registers. The row maximum is reduced warp ->
-// CTA (shared memory) -> cluster (distributed shared memory, two cluster
-// barriers), then each chunk goes through exp, the 8-lane block amax
-// butterfly, the block scale, rounding and packing, and leaves through a
-// per-warp staging slice. cols <= C*1024*16 = 131072 keys per row.
+// One thread-block cluster per row; the row is split into C <= 8 contiguous
+// runs of whole 32-key blocks, one run per CTA, one block per thread (read as
+// four 32-byte sectors). The row maximum is reduced thread -> warp -> CTA
+// (shared memory) -> cluster (distributed shared memory between two cluster
+// barriers); then each thread exponentiates its 32 keys with packed fp32x2
+// arithmetic and quantizes its block. cols <= C * 1024 * 32 = 262144 keys.
 #include <cooperative_groups.h>
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "mxq_block.cuh"
 #include "mxq_device.cuh"
 #include "mxq_internal.h"
 
@@ -25,56 +25,77 @@ namespace cg = cooperative_groups;
 
 namespace mxq {
 
-constexpr int kR = 4;            // 16-byte chunks per thread
-constexpr int kMaxCluster = 8;   // portable cluster size
+constexpr int kMaxCluster = 8;  // portable cluster size
 constexpr int kMaxThreads = 1024;
 
 // The library's own fp32 exponential (the same definition the CPU oracle
 // implements independently):
-//   t = RN(d * L2E), n = rint(t) (ties to even),
+//   t = RN(d * L2E), n = t rounded to an integer, ties to even,
 //   r = RN(d - n*LN2_HI) and r = RN(r - n*LN2_LO), both fused (Cody & Waite),
 //   p = Horner over 1/k!, k = 7..0, one fused multiply-add per step,
-//   e^d = p * 2^n (split in two exact-then-rounded products outside
-//   2^[-126,127]); t < -160 -> +0, t > 160 -> +inf, NaN -> NaN.
+//   e^d = p * 2^n (outside 2^[-126,127] as two exact-then-rounded products
+//   through 2^(n+-64)); t < -160 -> +0, t > 160 -> +inf, NaN -> NaN.
 // L2E = 1/ln2 and LN2_LO = ln2 - LN2_HI rounded to fp32, LN2_HI = ln 2 cut to
 // 16 significant bits, 1/k! rounded to fp32.
+constexpr float kL2E = 0x1.715476p+0f, kLn2Hi = 0x1.62e4p-1f, kLn2Lo = 0x1.7f7d1cp-20f;
+constexpr float kC0 = 0x1p+0f, kC1 = 0x1p+0f, kC2 = 0x1p-1f, kC3 = 0x1.555556p-3f, kC4 = 0x1.555556p-5f,
+                kC5 = 0x1.111112p-7f, kC6 = 0x1.6c16c2p-10f, kC7 = 0x1.a01a02p-13f;
+constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer (|x| < 2^22)
+
 __device__ __forceinline__ float pow2i(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
 
+// general form, any input
 __device__ __forceinline__ float expf_mxq(float d) {
-    const float L2E = 0x1.715476p+0f, LN2_HI = 0x1.62e4p-1f, LN2_LO = 0x1.7f7d1cp-20f;
     if (d != d) return d;
-    float t = __fmul_rn(d, L2E);
+    float t = __fmul_rn(d, kL2E);
     if (t < -160.0f) return 0.0f;
     if (t > 160.0f) return __uint_as_float(0x7F800000u);
-    float n = rintf(t);
-    float r = __fmaf_rn(-n, LN2_HI, d);
-    r = __fmaf_rn(-n, LN2_LO, r);
-    float p = 0x1.a01a02p-13f;
-    p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);
-    p = __fmaf_rn(p, r, 0x1.111112p-7f);
-    p = __fmaf_rn(p, r, 0x1.555556p-5f);
-    p = __fmaf_rn(p, r, 0x1.555556p-3f);
-    p = __fmaf_rn(p, r, 0x1p-1f);
-    p = __fmaf_rn(p, r, 0x1p+0f);
-    p = __fmaf_rn(p, r, 0x1p+0f);
+    float n = __fsub_rn(__fadd_rn(t, kRound), kRound);  // rint(t), ties to even
+    float r = __fmaf_rn(-n, kLn2Hi, d);
+    r = __fmaf_rn(-n, kLn2Lo, r);
+    float p = kC7;
+    p = __fmaf_rn(p, r, kC6);
+    p = __fmaf_rn(p, r, kC5);
+    p = __fmaf_rn(p, r, kC4);
+    p = __fmaf_rn(p, r, kC3);
+    p = __fmaf_rn(p, r, kC2);
+    p = __fmaf_rn(p, r, kC1);
+    p = __fmaf_rn(p, r, kC0);
     int ni = (int)n;
     if (ni < -126) return __fmul_rn(__fmul_rn(p, pow2i(ni + 64)), pow2i(-64));
     if (ni > 127) return __fmul_rn(__fmul_rn(p, pow2i(ni - 64)), pow2i(64));
     return __fmul_rn(p, pow2i(ni));
 }
 
+// Same function on a packed pair of shifted scores d = (lo, hi), valid when both
+// t = d*L2E lie in [-126, 127] (then 2^n is one normal fp32 and one product
+// suffices): n from the 1.5*2^23 add, 2^n's bits from that sum's bits.
+__device__ __forceinline__ unsigned long long expf_mxq2(unsigned long long d) {
+    const unsigned long long tm = f2add(f2mul(d, dup2(kL2E)), dup2(kRound));
+    const unsigned long long nn = f2sub(dup2(kRound), tm);  // -n, exact
+    unsigned long long r = f2fma(nn, dup2(kLn2Hi), d);
+    r = f2fma(nn, dup2(kLn2Lo), r);
+    unsigned long long p = f2fma(dup2(kC7), r, dup2(kC6));
+    p = f2fma(p, r, dup2(kC5));
+    p = f2fma(p, r, dup2(kC4));
+    p = f2fma(p, r, dup2(kC3));
+    p = f2fma(p, r, dup2(kC2));
+    p = f2fma(p, r, dup2(kC1));
+    p = f2fma(p, r, dup2(kC0));
+    float a, b;
+    upk(tm, a, b);
+    // bits(tm) = 0x4B400000 + n, so (n + 127) << 23 = bits(tm) * 2^23 + 0x3F800000 (mod 2^32)
+    const float sa = __uint_as_float(__float_as_uint(a) * 0x800000u + 0x3F800000u);
+    const float sb = __uint_as_float(__float_as_uint(b) * 0x800000u + 0x3F800000u);
+    return f2mul(p, pk(sa, sb));
+}
+
 template <int F>
-__global__ void __launch_bounds__(kMaxThreads) k_exp_quantize(const float* __restrict__ scores,
-                                                             uint8_t* __restrict__ codes,
-                                                             void* __restrict__ scales, long long cols) {
-    constexpr int W = Fmt<F>::W;
-    constexpr int LB = 4 * W / 8;  // code bytes per 16-byte chunk
-    constexpr int PB = payload<F>();
+__global__ void __launch_bounds__(kMaxThreads) k_exp_quantize(const float* __restrict__ scores, void* __restrict__ codes,
+                                                             void* __restrict__ scales, long long cols, bool a32) {
     __shared__ float wmax[32];
-    __shared__ int wnan[32];
     __shared__ float cta_max;
     __shared__ float row_max;
-    __shared__ __align__(16) uint8_t stage[32][32 * LB];
 
     cg::cluster_group cl = cg::this_cluster();
     const int C = (int)cl.num_blocks();
@@ -82,121 +103,95 @@ __global__ void __launch_bounds__(kMaxThreads) k_exp_quantize(const float* __res
     const long long row = blockIdx.x / C;
     const long long bpr = cols / 32;
     const long long b0 = (long long)c * bpr / C, b1 = (long long)(c + 1) * bpr / C;
-    const int nch = (int)(b1 - b0) * 8;  // chunks owned by this CTA
-    const float* s = scores + row * cols + b0 * 32;
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5, NT = blockDim.x;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const bool valid = t < (int)(b1 - b0);
+    const long long blk = row * bpr + b0 + t;  // this thread's block in the flat block space
     const float NEG_INF = __uint_as_float(0xFF800000u);
 
-    float x[kR][4];
-    float m = NEG_INF;
-    int nan = 0;
+    uint32_t w[32];
+    if (valid) {
+        load_block<float>(scores, blk, w, a32);
+    } else {
 #pragma unroll
-    for (int j = 0; j < kR; ++j) {
-        const int k = t + j * NT;
-        uint4 v = k < nch ? ld_stream_v4(s + 4 * k) : make_uint4(0xFF800000u, 0xFF800000u, 0xFF800000u, 0xFF800000u);
-        x[j][0] = __uint_as_float(v.x);
-        x[j][1] = __uint_as_float(v.y);
-        x[j][2] = __uint_as_float(v.z);
-        x[j][3] = __uint_as_float(v.w);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            nan |= x[j][i] != x[j][i];
-            m = fmaxf(m, x[j][i]);
-        }
+        for (int i = 0; i < 32; ++i) w[i] = 0xFF800000u;
     }
-    // row maximum: warp, CTA, cluster
+    // row maximum (NaN anywhere -> NaN): thread, warp, CTA, cluster
+    float m[11];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    nan = __any_sync(0xFFFFFFFFu, nan);
-    if (lane == 0) {
-        wmax[warp] = m;
-        wnan[warp] = nan;
-    }
+    for (int i = 0; i < 10; ++i)
+        m[i] = max3_nan(__uint_as_float(w[3 * i]), __uint_as_float(w[3 * i + 1]), __uint_as_float(w[3 * i + 2]));
+    m[10] = max_nan(__uint_as_float(w[30]), __uint_as_float(w[31]));
+    float mx = max3_nan(max3_nan(m[0], m[1], m[2]), max3_nan(m[3], m[4], m[5]), max3_nan(m[6], m[7], m[8]));
+    mx = max3_nan(mx, m[9], m[10]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = max_nan(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    if (lane == 0) wmax[warp] = mx;
     __syncthreads();
     if (warp == 0) {
-        const int nw = NT >> 5;
-        float mm = lane < nw ? wmax[lane] : NEG_INF;
-        int nn = lane < nw ? wnan[lane] : 0;
+        const int nw = blockDim.x >> 5;
+        float v = lane < nw ? wmax[lane] : NEG_INF;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xFFFFFFFFu, mm, o));
-        nn = __any_sync(0xFFFFFFFFu, nn);
-        if (lane == 0) cta_max = nn ? __uint_as_float(0x7FC00000u) : mm;
+        for (int o = 16; o > 0; o >>= 1) v = max_nan(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+        if (lane == 0) cta_max = v;
     }
     cl.sync();
     if (t == 0) {
-        float mm = NEG_INF;
-        int nn = 0;
-        for (int r = 0; r < C; ++r) {
-            float v = *cl.map_shared_rank(&cta_max, r);
-            nn |= v != v;
-            mm = fmaxf(mm, v);
-        }
-        row_max = nn ? __uint_as_float(0x7FC00000u) : mm;
+        float v = NEG_INF;
+        for (int r = 0; r < C; ++r) v = max_nan(v, *cl.map_shared_rank(&cta_max, r));
+        row_max = v;
     }
-    cl.sync();  // remote reads done before any CTA may exit; row_max visible
+    cl.sync();  // every remote read is done before any CTA may exit; row_max visible
+    if (!valid) return;
     const float mr = row_max;
 
-    uint8_t* st = stage[warp];
-    uint8_t* gcodes = codes + (row * bpr + b0) * PB;
+    // shifted scores, then e^d (fast packed path unless some t < -126 in this block)
+    float tmin = 0.0f;
 #pragma unroll
-    for (int j = 0; j < kR; ++j) {
-        const int k = t + j * NT;
-        float p[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) p[i] = expf_mxq(__fsub_rn(x[j][i], mr));
-        uint32_t am = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) am = max(am, __float_as_uint(p[i]) & 0x7FFFFFFFu);
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
-        const uint32_t byte = scale_byte<F>(am);
-        const float inv = inv_scale(byte);
-        mul2(p[0], p[1], inv);
-        mul2(p[2], p[3], inv);
-        uint32_t cw[1];
-        encode<F, 4>(p, cw);
-        uint32_t w = byte == 0xFFu ? 0u : cw[0];
-        if constexpr (W == 6) {
-            w = pack6x4(w);
-            st[lane * 3] = (uint8_t)w;
-            st[lane * 3 + 1] = (uint8_t)(w >> 8);
-            st[lane * 3 + 2] = (uint8_t)(w >> 16);
-        } else if constexpr (W == 4) {
-            *reinterpret_cast<uint16_t*>(st + lane * 2) = (uint16_t)w;
-        } else {
-            *reinterpret_cast<uint32_t*>(st + lane * 4) = w;
-        }
-        if ((lane & 7) == 0 && k < nch) {
-            const long long b = row * bpr + b0 + k / 8;
-            if constexpr (Fmt<F>::FIXED) reinterpret_cast<uint16_t*>(scales)[b] = (uint16_t)byte;
-            else reinterpret_cast<uint8_t*>(scales)[b] = (uint8_t)byte;
-        }
-        __syncwarp();
-        const int k0 = warp * 32 + j * NT;  // first chunk of this warp's row slice
-        const int nvalid = max(0, min(32, nch - k0));
-        const int nbytes = nvalid * LB;      // multiple of 8 (whole blocks)
-        if (8 * lane < nbytes)
-            *reinterpret_cast<uint2*>(gcodes + (long long)k0 * LB + 8 * lane) =
-                *reinterpret_cast<const uint2*>(st + 8 * lane);
-        __syncwarp();
+    for (int i = 0; i < 16; ++i) {
+        unsigned long long d = f2sub(pk(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1])), dup2(mr));
+        float a, b;
+        upk(d, a, b);
+        w[2 * i] = __float_as_uint(a);
+        w[2 * i + 1] = __float_as_uint(b);
+        tmin = fminf(tmin, fminf(a, b));
     }
+    if (__fmul_rn(tmin, kL2E) >= -126.0f) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float a, b;
+            upk(expf_mxq2(pk(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1]))), a, b);
+            w[2 * i] = __float_as_uint(a);
+            w[2 * i + 1] = __float_as_uint(b);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(expf_mxq(__uint_as_float(w[i])));
+    }
+    // p >= 0 (or NaN): bit patterns order like the values
+    uint32_t am = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) am = max(am, w[i] & 0x7FFFFFFFu);
+    const uint32_t byte = scale_byte<F>(am);
+    uint32_t out[8];
+    encode_block<F, float>(w, byte, out);
+    store_payload<F>(codes, blk, out, a32);
+    store_scale<F>(scales, blk, byte);
 }
 
-bool exp_quantize_supported(long long cols) { return cols > 0 && cols % 32 == 0 && cols <= 131072; }
+bool exp_quantize_supported(long long cols) { return cols > 0 && cols % 32 == 0 && cols <= 262144; }
 
 template <int F>
 static cudaError_t launch_xq(const float* scores, long long rows, long long cols, void* codes, void* scales,
                              cudaStream_t st) {
     const long long bpr = cols / 32;
-    int C = (int)((cols + 4095) / 4096);
+    long long C = (bpr + 127) / 128;  // about 128 blocks (4096 keys) per CTA
     if (C > kMaxCluster) C = kMaxCluster;
     if (C < 1) C = 1;
-    const long long max_blocks = (bpr + C - 1) / C;
-    const long long chunks = max_blocks * 8;
-    long long nt = (chunks + kR - 1) / kR;
-    nt = (nt + 31) / 32 * 32;
+    const long long per_cta = (bpr + C - 1) / C;
+    const long long nt = (per_cta + 31) / 32 * 32;
     if (nt > kMaxThreads) return cudaErrorNotSupported;
     if (rows * C > 0x7FFFFFFFLL) return cudaErrorNotSupported;
+    const bool a32 = ((reinterpret_cast<uintptr_t>(scores) | reinterpret_cast<uintptr_t>(codes)) & 31) == 0;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(rows * C), 1, 1);
@@ -210,7 +205,7 @@ static cudaError_t launch_xq(const float* scores, long long rows, long long cols
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_exp_quantize<F>, scores, reinterpret_cast<uint8_t*>(codes), scales, cols);
+    return cudaLaunchKernelEx(&cfg, k_exp_quantize<F>, scores, codes, scales, cols, a32);
 }
 
 cudaError_t launch_exp_quantize(int fmt, const float* scores, long long rows, long long cols, void* codes,

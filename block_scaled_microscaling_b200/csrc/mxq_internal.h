@@ -14,12 +14,12 @@ struct Seg {
     void* codes;
     void* scales;
     long long nblocks;  // blocks of 32 values
-    long long tile0;    // first warp tile of this tensor (filled by the launcher)
+    long long blk0;     // first block of this tensor in the concatenation (filled by the launcher)
 };
 template <int N> struct SegTable {
     Seg seg[N];
     int n;
-    long long ntiles;
+    long long nblocks;  // all tensors' blocks
 };
 
 // fmt: 0 AXS-6, 1 E2M3, 2 E3M2, 3 E4M3, 4 E2M1; dtype: 0 fp32, 1 bf16

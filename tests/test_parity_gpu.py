@@ -197,10 +197,10 @@ def test_errors_with_device_pointers():
     y = torch.zeros(4, 64, dtype=torch.bfloat16, device="cuda")
     assert mxq.mxq_fake_quantize(f, x.data_ptr(), 1, 4, 64, x.data_ptr(), st) == 0             # in place ok
     assert mxq.mxq_fake_quantize(f, x.data_ptr(), 1, 4, 64, x.data_ptr() + 64, st) == 1        # partial overlap
-    big = torch.zeros(1, 131072 + 32, dtype=torch.float32, device="cuda")
-    cb = torch.zeros(1, (131072 + 32) // 2, dtype=torch.uint8, device="cuda")
-    sb = torch.zeros(1, (131072 + 32) // 32, dtype=torch.uint8, device="cuda")
-    assert mxq.mxq_exp_quantize(4, big.data_ptr(), 1, 131072 + 32, cb.data_ptr(), sb.data_ptr(), st) == 4
+    big = torch.zeros(1, 262144 + 32, dtype=torch.float32, device="cuda")
+    cb = torch.zeros(1, (262144 + 32) // 2, dtype=torch.uint8, device="cuda")
+    sb = torch.zeros(1, (262144 + 32) // 32, dtype=torch.uint8, device="cuda")
+    assert mxq.mxq_exp_quantize(4, big.data_ptr(), 1, 262144 + 32, cb.data_ptr(), sb.data_ptr(), st) == 4
     torch.cuda.synchronize()
     del y
 
@@ -208,7 +208,7 @@ def test_errors_with_device_pointers():
 # ---- exp-then-quantize softmax stage --------------------------------------------------
 
 @pytest.mark.parametrize("fmt", FMTS)
-@pytest.mark.parametrize("cols", [32, 96, 1024, 4096, 4992, 32768, 131072])
+@pytest.mark.parametrize("cols", [32, 96, 1024, 4096, 4992, 32768, 131072, 262144])
 def test_exp_quantize_matches_oracle(fmt, cols):
     rows = max(2, min(64, 2 ** 21 // cols))
     s = synthetic.attention_scores(seed=4, heads=1, queries=rows, keys=cols)
