@@ -43,47 +43,132 @@ __device__ __forceinline__ int find_seg(const SegTable<NSEG>& tab, long long b) 
 // ---------------------------------------------------------------------------
 // kernels
 
+// Per-kernel shape choices, picked by measurement on B200 (median of repeated
+// graph timings over the five workloads): a thread keeps two blocks in flight
+// only in the grouped FP6 quantize (decoder layers, ~100M values per launch:
+// 0.92 vs 0.77-0.82 of HBM peak); one block elsewhere (a 47 MB launch loses
+// ~5% with two: fewer, longer threads). Shared-memory staging of 6-bit stores
+// helps single-tensor FP6 quantize (0.91 vs 0.79) but not AXS-6 or grouped.
+template <int F, typename T, int NSEG> __host__ __device__ constexpr int q_unroll() {
+    return (NSEG > 1 && Fmt<F>::W == 6 && !Fmt<F>::FIXED && sizeof(T) == 2) ? 2 : 1;
+}
+template <int F, typename T, int NSEG> __host__ __device__ constexpr bool q_stage() {
+    return NSEG == 1 && Fmt<F>::W == 6 && !Fmt<F>::FIXED;
+}
+
+// 6-bit payloads are 24 bytes: a warp's 32 consecutive blocks are assembled in
+// shared memory and leave as 16-byte stores (48 of them) instead of 3 x 8 bytes
+// per thread.
+template <int F>
+__device__ __forceinline__ void warp_store6(void* codes, long long first_blk, int nvalid, const uint32_t* out,
+                                            uint8_t* stage, int lane) {
+    uint2* q = reinterpret_cast<uint2*>(stage + 24 * lane);
+    q[0] = make_uint2(out[0], out[1]);
+    q[1] = make_uint2(out[2], out[3]);
+    q[2] = make_uint2(out[4], out[5]);
+    __syncwarp();
+    char* g = reinterpret_cast<char*>(codes) + first_blk * 24;
+    const int nbytes = 24 * nvalid;
+    for (int i = 16 * lane; i + 16 <= nbytes; i += 512)
+        st_stream_v4(g + i, *reinterpret_cast<const uint4*>(stage + i));
+    if ((nbytes & 15) && lane == 0) *reinterpret_cast<uint2*>(g + (nbytes & ~15)) = *reinterpret_cast<const uint2*>(stage + (nbytes & ~15));
+    __syncwarp();
+}
+
 template <int F, typename T, int NSEG>
 __global__ void __launch_bounds__(kThreads) k_quantize(const __grid_constant__ SegTable<NSEG> tab) {
+    constexpr int U = q_unroll<F, T, NSEG>();
+    constexpr bool STAGE = q_stage<F, T, NSEG>();
+    __shared__ __align__(16) uint8_t stage[STAGE ? kThreads / 32 : 1][STAGE ? 32 * 24 : 16];
+    const int lane = threadIdx.x & 31;
     const long long stride = (long long)gridDim.x * kThreads;
-    for (long long gb = (long long)blockIdx.x * kThreads + threadIdx.x; gb < tab.nblocks; gb += stride) {
-        const Seg& g = tab.seg[find_seg(tab, gb)];
-        const long long b = gb - g.blk0;
-        const bool a32 = ((reinterpret_cast<uintptr_t>(g.src) | reinterpret_cast<uintptr_t>(g.codes)) & 31) == 0;
-        uint32_t w[Blk<T>::NW];
-        load_block<T>(g.src, b, w, a32);
-        const uint32_t byte = scale_byte<F>(block_amax<T>(w));
-        uint32_t out[8];
-        encode_block<F, T>(w, byte, out);
-        store_payload<F>(g.codes, b, out, a32);
-        store_scale<F>(g.scales, b, byte);
+    const long long N = tab.nblocks;
+    // warp-uniform trip count: every lane of a warp takes the same iterations
+    for (long long base = (long long)blockIdx.x * kThreads + (threadIdx.x & ~31); base < N; base += U * stride) {
+        uint32_t w[U][Blk<T>::NW];
+        const Seg* g[U];
+        long long b[U];
+        bool a32[U], ok[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long gb = base + u * stride + lane;
+            ok[u] = gb < N;
+            g[u] = &tab.seg[find_seg(tab, ok[u] ? gb : 0)];
+            b[u] = gb - g[u]->blk0;
+            a32[u] = ((reinterpret_cast<uintptr_t>(g[u]->src) | reinterpret_cast<uintptr_t>(g[u]->codes)) & 31) == 0;
+            if (ok[u]) load_block<T>(g[u]->src, b[u], w[u], a32[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint32_t byte = scale_byte<F>(block_amax<T>(w[u]));
+            uint32_t out[8];
+            encode_block<F, T>(w[u], byte, out);
+            if constexpr (STAGE) {
+                // whole warp in one tensor: staged 16-byte stores; else per thread
+                const long long first = base + u * stride;  // lane 0's block, warp-uniform
+                const int nvalid = (int)min(32LL, N - first);
+                const Seg* g0 = &tab.seg[find_seg(tab, first < N ? first : 0)];
+                const bool same = __all_sync(0xFFFFFFFFu, !ok[u] || g[u] == g0);
+                if (nvalid > 0 && same) {
+                    warp_store6<F>(g0->codes, first - g0->blk0, nvalid, out, stage[threadIdx.x >> 5], lane);
+                } else if (ok[u]) {
+                    store_payload<F>(g[u]->codes, b[u], out, a32[u]);
+                }
+            } else {
+                if (ok[u]) store_payload<F>(g[u]->codes, b[u], out, a32[u]);
+            }
+            if (ok[u]) store_scale<F>(g[u]->scales, b[u], byte);
+        }
     }
 }
 
 template <int F, typename T>
 __global__ void __launch_bounds__(kThreads) k_dequantize(const void* __restrict__ codes, const void* __restrict__ scales,
                                                          void* __restrict__ dst, long long nblocks, bool a32) {
+    constexpr int U = 1;
     const long long stride = (long long)gridDim.x * kThreads;
-    for (long long b = (long long)blockIdx.x * kThreads + threadIdx.x; b < nblocks; b += stride) {
-        uint32_t pw[8];
-        load_payload<F>(codes, b, pw, a32);
-        const uint32_t byte = load_scale<F>(scales, b);
-        uint32_t o[Blk<T>::NW];
-        decode_block<F, T>(pw, byte, o);
-        store_block<T>(dst, b, o, a32);
+    for (long long base = (long long)blockIdx.x * kThreads + threadIdx.x; base < nblocks; base += U * stride) {
+        uint32_t pw[U][8];
+        uint32_t byte[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long b = base + u * stride;
+            if (b < nblocks) {
+                load_payload<F>(codes, b, pw[u], a32);
+                byte[u] = load_scale<F>(scales, b);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long b = base + u * stride;
+            if (b < nblocks) {
+                uint32_t o[Blk<T>::NW];
+                decode_block<F, T>(pw[u], byte[u], o);
+                store_block<T>(dst, b, o, a32);
+            }
+        }
     }
 }
 
 template <int F, typename T>
 __global__ void __launch_bounds__(kThreads) k_fake_quantize(const void* src, void* dst, long long nblocks, bool a32) {
+    constexpr int U = 1;
     const long long stride = (long long)gridDim.x * kThreads;
-    for (long long b = (long long)blockIdx.x * kThreads + threadIdx.x; b < nblocks; b += stride) {
-        uint32_t w[Blk<T>::NW];
-        load_block<T>(src, b, w, a32);
-        const uint32_t byte = scale_byte<F>(block_amax<T>(w));
-        uint32_t o[Blk<T>::NW];
-        fake_block<F, T>(w, byte, o);
-        store_block<T>(dst, b, o, a32);
+    for (long long base = (long long)blockIdx.x * kThreads + threadIdx.x; base < nblocks; base += U * stride) {
+        uint32_t w[U][Blk<T>::NW];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (base + u * stride < nblocks) load_block<T>(src, base + u * stride, w[u], a32);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long b = base + u * stride;
+            if (b < nblocks) {
+                const uint32_t byte = scale_byte<F>(block_amax<T>(w[u]));
+                uint32_t o[Blk<T>::NW];
+                fake_block<F, T>(w[u], byte, o);
+                store_block<T>(dst, b, o, a32);
+            }
+        }
     }
 }
 
@@ -112,6 +197,7 @@ static int grid_for(K kernel, long long nblocks) {
     int dev = 0;
     cudaGetDevice(&dev);
     long long cap = resident_ctas(reinterpret_cast<const void*>(kernel), dev);
+    // fill every SM first; a thread then takes its blocks U at a time
     long long want = (nblocks + kThreads - 1) / kThreads;
     return (int)(want < cap ? (want > 0 ? want : 1) : cap);
 }

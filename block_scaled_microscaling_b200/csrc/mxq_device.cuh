@@ -140,6 +140,14 @@ __device__ __forceinline__ float absmax_f32(float a, float b) {
 }
 
 // ---------------------------------------------------------------------------
+// cluster barrier without the release fence on every thread: only the thread
+// that published data for other CTAs orders it (fence.acq_rel.cluster), so the
+// barrier does not wait for every thread's loads and stores still in flight.
+__device__ __forceinline__ void cluster_publish_fence() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+__device__ __forceinline__ void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // the shared scale
 
 // |x| bit patterns order as unsigned integers: finite < +Inf < NaN.

@@ -7,12 +7,15 @@
 // an exponent-only scale from each 32-key block's maximum. Here the block is
 // never materialized: scores are read once and probabilities live in registers.
 //
-// One thread-block cluster per row; the row is split into C <= 8 contiguous
-// runs of whole 32-key blocks, one run per CTA, one block per thread (read as
-// four 32-byte sectors). The row maximum is reduced thread -> warp -> CTA
-// (shared memory) -> cluster (distributed shared memory between two cluster
-// barriers); then each thread exponentiates its 32 keys with packed fp32x2
-// arithmetic and quantizes its block. cols <= C * 1024 * 32 = 262144 keys.
+// A thread-block cluster works on one row at a time; the row is split into
+// C contiguous runs of whole 32-key blocks, one run per CTA, one block per
+// thread (read as four 32-byte sectors). Clusters are persistent: each walks
+// rows with a stride, prefetching its next row's blocks into a second register
+// buffer while the current row is reduced and quantized. The row maximum goes
+// thread -> warp -> CTA (shared memory) -> cluster (distributed shared memory,
+// one cluster barrier per row); then each thread exponentiates its 32 keys with
+// packed fp32x2 arithmetic and quantizes its block. C <= 8 (portable cluster)
+// for rows up to 131072 keys, 16 (non-portable) up to 262144.
 #include <cooperative_groups.h>
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -25,8 +28,7 @@ namespace cg = cooperative_groups;
 
 namespace mxq {
 
-constexpr int kMaxCluster = 8;  // portable cluster size
-constexpr int kMaxThreads = 1024;
+constexpr int kMaxThreads = 512;  // two 32-value register buffers per thread need <= 128 registers
 
 // The library's own fp32 exponential (the same definition the CPU oracle
 // implements independently):
@@ -90,39 +92,27 @@ __device__ __forceinline__ unsigned long long expf_mxq2(unsigned long long d) {
     return f2mul(p, pk(sa, sb));
 }
 
+// One row's work for one CTA once its block is in registers: row maximum
+// through the cluster, then exp + quantize of the thread's block. `it` picks
+// the maximum slot (double-buffered, so one cluster barrier per row suffices:
+// a CTA can write slot it&1 again only after the next row's barrier, which
+// every CTA reaches after its reads of this row's slots).
 template <int F>
-__global__ void __launch_bounds__(kMaxThreads) k_exp_quantize(const float* __restrict__ scores, void* __restrict__ codes,
-                                                             void* __restrict__ scales, long long cols, bool a32) {
-    __shared__ float wmax[32];
-    __shared__ float cta_max;
-    __shared__ float row_max;
-
-    cg::cluster_group cl = cg::this_cluster();
-    const int C = (int)cl.num_blocks();
-    const int c = (int)cl.block_rank();
-    const long long row = blockIdx.x / C;
-    const long long bpr = cols / 32;
-    const long long b0 = (long long)c * bpr / C, b1 = (long long)(c + 1) * bpr / C;
+__device__ __forceinline__ void exp_row(uint32_t (&w)[32], bool valid, long long blk, int it, int C,
+                                        cg::cluster_group& cl, float* wmax, float* slot, float* row_max,
+                                        void* codes, void* scales, bool a32) {
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const bool valid = t < (int)(b1 - b0);
-    const long long blk = row * bpr + b0 + t;  // this thread's block in the flat block space
     const float NEG_INF = __uint_as_float(0xFF800000u);
-
-    uint32_t w[32];
+    float mx = NEG_INF;
     if (valid) {
-        load_block<float>(scores, blk, w, a32);
-    } else {
+        float m[11];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) w[i] = 0xFF800000u;
+        for (int i = 0; i < 10; ++i)
+            m[i] = max3_nan(__uint_as_float(w[3 * i]), __uint_as_float(w[3 * i + 1]), __uint_as_float(w[3 * i + 2]));
+        m[10] = max_nan(__uint_as_float(w[30]), __uint_as_float(w[31]));
+        mx = max3_nan(max3_nan(m[0], m[1], m[2]), max3_nan(m[3], m[4], m[5]), max3_nan(m[6], m[7], m[8]));
+        mx = max3_nan(mx, m[9], m[10]);
     }
-    // row maximum (NaN anywhere -> NaN): thread, warp, CTA, cluster
-    float m[11];
-#pragma unroll
-    for (int i = 0; i < 10; ++i)
-        m[i] = max3_nan(__uint_as_float(w[3 * i]), __uint_as_float(w[3 * i + 1]), __uint_as_float(w[3 * i + 2]));
-    m[10] = max_nan(__uint_as_float(w[30]), __uint_as_float(w[31]));
-    float mx = max3_nan(max3_nan(m[0], m[1], m[2]), max3_nan(m[3], m[4], m[5]), max3_nan(m[6], m[7], m[8]));
-    mx = max3_nan(mx, m[9], m[10]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = max_nan(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
     if (lane == 0) wmax[warp] = mx;
@@ -132,19 +122,24 @@ __global__ void __launch_bounds__(kMaxThreads) k_exp_quantize(const float* __res
         float v = lane < nw ? wmax[lane] : NEG_INF;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v = max_nan(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-        if (lane == 0) cta_max = v;
+        if (lane == 0) {
+            slot[it & 1] = v;
+            cluster_publish_fence();
+        }
     }
-    cl.sync();
-    if (t == 0) {
-        float v = NEG_INF;
-        for (int r = 0; r < C; ++r) v = max_nan(v, *cl.map_shared_rank(&cta_max, r));
-        row_max = v;
+    cluster_arrive_relaxed();
+    cluster_wait();
+    if (warp == 0) {  // the C remote maxima, read in parallel by lanes 0..C-1
+        float v = lane < C ? cl.map_shared_rank(slot, lane)[it & 1] : NEG_INF;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v = max_nan(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+        if (lane == 0) *row_max = v;
     }
-    cl.sync();  // every remote read is done before any CTA may exit; row_max visible
+    __syncthreads();
     if (!valid) return;
-    const float mr = row_max;
+    const float mr = *row_max;
 
-    // shifted scores, then e^d (fast packed path unless some t < -126 in this block)
+    // shifted scores, then e^d (packed path unless some t < -126 in this block)
     float tmin = 0.0f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -167,15 +162,56 @@ __global__ void __launch_bounds__(kMaxThreads) k_exp_quantize(const float* __res
 #pragma unroll
         for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(expf_mxq(__uint_as_float(w[i])));
     }
-    // p >= 0 (or NaN): bit patterns order like the values
-    uint32_t am = 0;
+    // p >= 0 or NaN: a NaN-propagating max gives the block maximum (or NaN)
+    float q[11];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) am = max(am, w[i] & 0x7FFFFFFFu);
-    const uint32_t byte = scale_byte<F>(am);
+    for (int i = 0; i < 10; ++i) q[i] = max3_nan(__uint_as_float(w[3 * i]), __uint_as_float(w[3 * i + 1]), __uint_as_float(w[3 * i + 2]));
+    q[10] = max_nan(__uint_as_float(w[30]), __uint_as_float(w[31]));
+    float pm = max3_nan(max3_nan(q[0], q[1], q[2]), max3_nan(q[3], q[4], q[5]), max3_nan(q[6], q[7], q[8]));
+    pm = max3_nan(pm, q[9], q[10]);
+    const uint32_t byte = scale_byte<F>(__float_as_uint(pm) & 0x7FFFFFFFu);
     uint32_t out[8];
     encode_block<F, float>(w, byte, out);
     store_payload<F>(codes, blk, out, a32);
     store_scale<F>(scales, blk, byte);
+}
+
+// Persistent clusters: cluster k handles rows k, k + G, k + 2G, ...; each
+// thread prefetches its block of the next row into a second register buffer
+// while the current row is reduced and quantized.
+template <int F>
+__global__ void __launch_bounds__(kMaxThreads) k_exp_quantize(const float* __restrict__ scores, void* __restrict__ codes,
+                                                             void* __restrict__ scales, long long rows, long long cols,
+                                                             bool a32) {
+    __shared__ float wmax[32];
+    __shared__ float slot[2];
+    __shared__ float row_max;
+
+    cg::cluster_group cl = cg::this_cluster();
+    const int C = (int)cl.num_blocks();
+    const int c = (int)cl.block_rank();
+    const long long G = gridDim.x / C;
+    const long long bpr = cols / 32;
+    const long long b0 = (long long)c * bpr / C, b1 = (long long)(c + 1) * bpr / C;
+    const bool valid = (long long)threadIdx.x < b1 - b0;
+    const long long col_blk = b0 + threadIdx.x;
+
+    long long r = blockIdx.x / C;
+    uint32_t A[32], B[32];
+    if (valid && r < rows) load_block<float>(scores, r * bpr + col_blk, A, a32);
+    int it = 0;
+    while (r < rows) {
+        if (valid && r + G < rows) load_block<float>(scores, (r + G) * bpr + col_blk, B, a32);
+        exp_row<F>(A, valid, r * bpr + col_blk, it, C, cl, wmax, slot, &row_max, codes, scales, a32);
+        r += G;
+        ++it;
+        if (r >= rows) break;
+        if (valid && r + G < rows) load_block<float>(scores, (r + G) * bpr + col_blk, A, a32);
+        exp_row<F>(B, valid, r * bpr + col_blk, it, C, cl, wmax, slot, &row_max, codes, scales, a32);
+        r += G;
+        ++it;
+    }
+    cl.sync();  // no CTA leaves while another may still read its slots
 }
 
 bool exp_quantize_supported(long long cols) { return cols > 0 && cols % 32 == 0 && cols <= 262144; }
@@ -185,16 +221,15 @@ static cudaError_t launch_xq(const float* scores, long long rows, long long cols
                              cudaStream_t st) {
     const long long bpr = cols / 32;
     long long C = (bpr + 127) / 128;  // about 128 blocks (4096 keys) per CTA
-    if (C > kMaxCluster) C = kMaxCluster;
+    if (C > 8) C = 8;                 // portable cluster size
     if (C < 1) C = 1;
+    if ((bpr + C - 1) / C > kMaxThreads) C = 16;  // non-portable size, long rows only
     const long long per_cta = (bpr + C - 1) / C;
     const long long nt = (per_cta + 31) / 32 * 32;
     if (nt > kMaxThreads) return cudaErrorNotSupported;
-    if (rows * C > 0x7FFFFFFFLL) return cudaErrorNotSupported;
     const bool a32 = ((reinterpret_cast<uintptr_t>(scores) | reinterpret_cast<uintptr_t>(codes)) & 31) == 0;
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(rows * C), 1, 1);
     cfg.blockDim = dim3((unsigned)nt, 1, 1);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
@@ -205,7 +240,20 @@ static cudaError_t launch_xq(const float* scores, long long rows, long long cols
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_exp_quantize<F>, scores, codes, scales, cols, a32);
+    if (C > 8) {
+        cudaError_t e = cudaFuncSetAttribute(k_exp_quantize<F>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    // as many clusters as fit on the GPU at once (each then loops over rows)
+    cfg.gridDim = dim3((unsigned)(C * 1024), 1, 1);
+    int active = 0;
+    if (cudaOccupancyMaxActiveClusters(&active, k_exp_quantize<F>, &cfg) != cudaSuccess || active < 1) {
+        cudaGetLastError();
+        active = 148;
+    }
+    long long G = rows < active ? rows : active;
+    cfg.gridDim = dim3((unsigned)(G * C), 1, 1);
+    return cudaLaunchKernelEx(&cfg, k_exp_quantize<F>, scores, codes, scales, rows, cols, a32);
 }
 
 cudaError_t launch_exp_quantize(int fmt, const float* scores, long long rows, long long cols, void* codes,
