@@ -50,6 +50,29 @@ def peaks():
     return FALLBACK_HBM, "fallback"
 
 
+def ncu_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture, or None when
+    the kernel sources have changed since that capture (or it was not captured)."""
+    import glob
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    csrc = os.path.join(ROOT, "block_scaled_microscaling_b200", "csrc")
+    h = hashlib.sha256()
+    for fn in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")) +
+                     glob.glob(os.path.join(csrc, "*.h"))):
+        h.update(os.path.basename(fn).encode())
+        with open(fn, "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != d.get("csrc_sha256"):
+        return None
+    v = d.get("bytes_per_launch", {}).get(kernel)
+    return int(v) if v is not None else None
+
+
 def nbytes_q(fmt, n_elems, in_bytes):
     """Algorithmic bytes of one quantize (or dequantize) of n_elems values."""
     bits = {"axs6": 6, "mxfp6_e2m3": 6, "mxfp6_e3m2": 6, "mxfp8": 8, "mxfp4": 4}[fmt]
@@ -504,7 +527,7 @@ def main():
         "per_op": {nm: {"ms": round(v, 5), "GB/s": round(op_bytes / (v * 1e-3) / 1e9, 1),
                         "frac_hbm": round(op_bytes / (v * 1e-3) / 1e9 / hbm, 4)} for nm, v in op_ms.items()},
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": round(ach, 1), "peak": hbm,
-                     "peak_source": how, "unit": "GB/s", "frac": round(ach / hbm, 4), "traffic": None,
+                     "peak_source": how, "unit": "GB/s", "frac": round(ach / hbm, 4), "traffic": ncu_traffic(dominant),
                      "algorithmic_bytes_per_launch": op_bytes},
         "clocks": clk.summary(),
         "gpu_launches": 4 * args.steps,
