@@ -101,12 +101,20 @@ __device__ __forceinline__ void encode_block(const uint32_t* w, uint32_t byte, u
         }
     } else if constexpr (Fmt<F>::W == 8) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) out[j] = (code_pair<F, T>(w, 2 * j, inv) | (code_pair<F, T>(w, 2 * j + 1, inv) << 16)) & keep;
+        for (int j = 0; j < 8; ++j) {
+            float a0, a1, a2, a3;
+            upk(f2mul(pair<T>(w, 2 * j), dup2(inv)), a0, a1);
+            upk(f2mul(pair<T>(w, 2 * j + 1), dup2(inv)), a2, a3);
+            out[j] = cvt4_e4m3(a0, a1, a2, a3) & keep;
+        }
     } else {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-            out[j] = (code_pair<F, T>(w, 4 * j, inv) | (code_pair<F, T>(w, 4 * j + 1, inv) << 8) |
-                      (code_pair<F, T>(w, 4 * j + 2, inv) << 16) | (code_pair<F, T>(w, 4 * j + 3, inv) << 24)) & keep;
+        for (int j = 0; j < 4; ++j) {
+            float a[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) upk(f2mul(pair<T>(w, 4 * j + q), dup2(inv)), a[2 * q], a[2 * q + 1]);
+            out[j] = cvt8_e2m1(a[0], a[1], a[2], a[3], a[4], a[5], a[6], a[7]) & keep;
+        }
     }
 }
 
@@ -221,5 +229,6 @@ __device__ __forceinline__ void fake_block(const uint32_t* w, uint32_t byte, uin
     encode_block<F, T>(w, byte, pw);
     decode_block<F, T>(pw, byte, o);
 }
+
 
 }  // namespace mxq

@@ -55,6 +55,13 @@ __device__ __forceinline__ void st_v8(void* p, const uint32_t* r) {
                  :: "l"(p), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
                  : "memory");
 }
+// 32-byte loads with an L2 priority hint: keep (first pass over data that is
+// read again soon) or drop first (last use)
+__device__ __forceinline__ void ld_v8_keep(const void* p, uint32_t* r) {
+    asm volatile("ld.global.nc.L1::no_allocate.L2::evict_last.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "l"(p));
+}
 // 16-byte halves through L1 (the second half of a sector then hits L1); p 16-byte aligned
 __device__ __forceinline__ void ld_2v4(const void* p, uint32_t* r) {
     uint4 a, b;
@@ -127,6 +134,12 @@ __device__ __forceinline__ float max3_nan(float a, float b, float c) {
     asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
 }
+// three-input minimum (a NaN operand is ignored)
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
 // max(|a|, |b|) of two bf16 pairs, lane-wise; NaN -> NaN (sign bits of the result are not meaningful)
 __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
     uint32_t r;
@@ -138,14 +151,6 @@ __device__ __forceinline__ float absmax_f32(float a, float b) {
     asm("max.NaN.xorsign.abs.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
     return r;
 }
-
-// ---------------------------------------------------------------------------
-// cluster barrier without the release fence on every thread: only the thread
-// that published data for other CTAs orders it (fence.acq_rel.cluster), so the
-// barrier does not wait for every thread's loads and stores still in flight.
-__device__ __forceinline__ void cluster_publish_fence() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
-__device__ __forceinline__ void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory"); }
-__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // the shared scale
@@ -195,6 +200,31 @@ template <> __device__ __forceinline__ uint32_t cvt2<F_E2M1>(float lo, float hi)
     asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u32.u8 %0, t; }"
         : "=r"(r) : "f"(hi), "f"(lo));
     return r;
+}
+
+// Eight values -> one word of eight E2M1 codes (nibble k = code of value k):
+// four conversions straight into byte registers, one vector move.
+__device__ __forceinline__ uint32_t cvt8_e2m1(float v0, float v1, float v2, float v3, float v4, float v5, float v6,
+                                              float v7) {
+    uint32_t w;
+    asm("{ .reg .b8 b0, b1, b2, b3;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n"
+        "mov.b32 %0, {b0, b1, b2, b3}; }"
+        : "=r"(w) : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+    return w;
+}
+// Four values -> one word of four E4M3 codes (byte k = code of value k).
+__device__ __forceinline__ uint32_t cvt4_e4m3(float v0, float v1, float v2, float v3) {
+    uint32_t w;
+    asm("{ .reg .b16 h0, h1;\n"
+        "cvt.rn.satfinite.e4m3x2.f32 h0, %2, %1;\n"
+        "cvt.rn.satfinite.e4m3x2.f32 h1, %4, %3;\n"
+        "mov.b32 %0, {h0, h1}; }"
+        : "=r"(w) : "f"(v0), "f"(v1), "f"(v2), "f"(v3));
+    return w;
 }
 
 // AXS-6 code of x (already multiplied by 2^-Es): sign | min(rne(16|x|), 31).

@@ -7,16 +7,11 @@
 // an exponent-only scale from each 32-key block's maximum. Here the block is
 // never materialized: scores are read once and probabilities live in registers.
 //
-// A thread-block cluster works on one row at a time; the row is split into
-// C contiguous runs of whole 32-key blocks, one run per CTA, one block per
-// thread (read as four 32-byte sectors). Clusters are persistent: each walks
-// rows with a stride, prefetching its next row's blocks into a second register
-// buffer while the current row is reduced and quantized. The row maximum goes
-// thread -> warp -> CTA (shared memory) -> cluster (distributed shared memory,
-// one cluster barrier per row); then each thread exponentiates its 32 keys with
-// packed fp32x2 arithmetic and quantizes its block. C <= 8 (portable cluster)
-// for rows up to 131072 keys, 16 (non-portable) up to 262144.
-#include <cooperative_groups.h>
+// One CTA per row (32 to 1024 threads, two to four blocks each), two passes: the
+// first streams the row from HBM for its maximum with loads marked to stay in
+// L2, the second re-reads it from L2 and exponentiates and quantizes each
+// 32-key block in registers. The launcher keeps the rows in flight within half
+// of L2, so HBM sees each score once. Any row length (cols % 32 == 0).
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -24,11 +19,8 @@
 #include "mxq_device.cuh"
 #include "mxq_internal.h"
 
-namespace cg = cooperative_groups;
-
 namespace mxq {
 
-constexpr int kMaxThreads = 512;  // two 32-value register buffers per thread need <= 128 registers
 
 // The library's own fp32 exponential (the same definition the CPU oracle
 // implements independently):
@@ -92,67 +84,22 @@ __device__ __forceinline__ unsigned long long expf_mxq2(unsigned long long d) {
     return f2mul(p, pk(sa, sb));
 }
 
-// One row's work for one CTA once its block is in registers: row maximum
-// through the cluster, then exp + quantize of the thread's block. `it` picks
-// the maximum slot (double-buffered, so one cluster barrier per row suffices:
-// a CTA can write slot it&1 again only after the next row's barrier, which
-// every CTA reaches after its reads of this row's slots).
-template <int F>
-__device__ __forceinline__ void exp_row(uint32_t (&w)[32], bool valid, long long blk, int it, int C,
-                                        cg::cluster_group& cl, float* wmax, float* slot, float* row_max,
-                                        void* codes, void* scales, bool a32) {
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const float NEG_INF = __uint_as_float(0xFF800000u);
-    float mx = NEG_INF;
-    if (valid) {
-        float m[11];
-#pragma unroll
-        for (int i = 0; i < 10; ++i)
-            m[i] = max3_nan(__uint_as_float(w[3 * i]), __uint_as_float(w[3 * i + 1]), __uint_as_float(w[3 * i + 2]));
-        m[10] = max_nan(__uint_as_float(w[30]), __uint_as_float(w[31]));
-        mx = max3_nan(max3_nan(m[0], m[1], m[2]), max3_nan(m[3], m[4], m[5]), max3_nan(m[6], m[7], m[8]));
-        mx = max3_nan(mx, m[9], m[10]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = max_nan(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-    if (lane == 0) wmax[warp] = mx;
-    __syncthreads();
-    if (warp == 0) {
-        const int nw = blockDim.x >> 5;
-        float v = lane < nw ? wmax[lane] : NEG_INF;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v = max_nan(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-        if (lane == 0) {
-            slot[it & 1] = v;
-            cluster_publish_fence();
-        }
-    }
-    cluster_arrive_relaxed();
-    cluster_wait();
-    if (warp == 0) {  // the C remote maxima, read in parallel by lanes 0..C-1
-        float v = lane < C ? cl.map_shared_rank(slot, lane)[it & 1] : NEG_INF;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v = max_nan(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-        if (lane == 0) *row_max = v;
-    }
-    __syncthreads();
-    if (!valid) return;
-    const float mr = *row_max;
-
-    // shifted scores, then e^d (packed path unless some t < -126 in this block)
+// Shifted scores d = x - mr -> e^d, in place, for n values (n even); packed
+// path unless some t = d*L2E < -126 among them.
+template <int N>
+__device__ __forceinline__ void exp_values(uint32_t (&w)[N], float mr) {
     float tmin = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        unsigned long long d = f2sub(pk(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1])), dup2(mr));
+    for (int i = 0; i < N / 2; ++i) {
         float a, b;
-        upk(d, a, b);
+        upk(f2sub(pk(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1])), dup2(mr)), a, b);
         w[2 * i] = __float_as_uint(a);
         w[2 * i + 1] = __float_as_uint(b);
-        tmin = fminf(tmin, fminf(a, b));
+        tmin = min3f(tmin, a, b);
     }
     if (__fmul_rn(tmin, kL2E) >= -126.0f) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < N / 2; ++i) {
             float a, b;
             upk(expf_mxq2(pk(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1]))), a, b);
             w[2 * i] = __float_as_uint(a);
@@ -160,15 +107,21 @@ __device__ __forceinline__ void exp_row(uint32_t (&w)[32], bool valid, long long
         }
     } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(expf_mxq(__uint_as_float(w[i])));
+        for (int i = 0; i < N; ++i) w[i] = __float_as_uint(expf_mxq(__uint_as_float(w[i])));
     }
-    // p >= 0 or NaN: a NaN-propagating max gives the block maximum (or NaN)
+}
+
+
+template <int F>
+__device__ __forceinline__ void exp_quant_block(uint32_t (&w)[32], float mr, long long blk, void* codes, void* scales,
+                                                bool a32) {
+    exp_values<32>(w, mr);
     float q[11];
 #pragma unroll
     for (int i = 0; i < 10; ++i) q[i] = max3_nan(__uint_as_float(w[3 * i]), __uint_as_float(w[3 * i + 1]), __uint_as_float(w[3 * i + 2]));
     q[10] = max_nan(__uint_as_float(w[30]), __uint_as_float(w[31]));
     float pm = max3_nan(max3_nan(q[0], q[1], q[2]), max3_nan(q[3], q[4], q[5]), max3_nan(q[6], q[7], q[8]));
-    pm = max3_nan(pm, q[9], q[10]);
+    pm = max3_nan(pm, q[9], q[10]);  // p >= 0 or NaN: the block maximum (or NaN)
     const uint32_t byte = scale_byte<F>(__float_as_uint(pm) & 0x7FFFFFFFu);
     uint32_t out[8];
     encode_block<F, float>(w, byte, out);
@@ -176,84 +129,116 @@ __device__ __forceinline__ void exp_row(uint32_t (&w)[32], bool valid, long long
     store_scale<F>(scales, blk, byte);
 }
 
-// Persistent clusters: cluster k handles rows k, k + G, k + 2G, ...; each
-// thread prefetches its block of the next row into a second register buffer
-// while the current row is reduced and quantized.
-template <int F>
-__global__ void __launch_bounds__(kMaxThreads) k_exp_quantize(const float* __restrict__ scores, void* __restrict__ codes,
-                                                             void* __restrict__ scales, long long rows, long long cols,
-                                                             bool a32) {
-    __shared__ float wmax[32];
-    __shared__ float slot[2];
-    __shared__ float row_max;
-
-    cg::cluster_group cl = cg::this_cluster();
-    const int C = (int)cl.num_blocks();
-    const int c = (int)cl.block_rank();
-    const long long G = gridDim.x / C;
-    const long long bpr = cols / 32;
-    const long long b0 = (long long)c * bpr / C, b1 = (long long)(c + 1) * bpr / C;
-    const bool valid = (long long)threadIdx.x < b1 - b0;
-    const long long col_blk = b0 + threadIdx.x;
-
-    long long r = blockIdx.x / C;
-    uint32_t A[32], B[32];
-    if (valid && r < rows) load_block<float>(scores, r * bpr + col_blk, A, a32);
-    int it = 0;
-    while (r < rows) {
-        if (valid && r + G < rows) load_block<float>(scores, (r + G) * bpr + col_blk, B, a32);
-        exp_row<F>(A, valid, r * bpr + col_blk, it, C, cl, wmax, slot, &row_max, codes, scales, a32);
-        r += G;
-        ++it;
-        if (r >= rows) break;
-        if (valid && r + G < rows) load_block<float>(scores, (r + G) * bpr + col_blk, A, a32);
-        exp_row<F>(B, valid, r * bpr + col_blk, it, C, cl, wmax, slot, &row_max, codes, scales, a32);
-        r += G;
-        ++it;
-    }
-    cl.sync();  // no CTA leaves while another may still read its slots
+__device__ __forceinline__ float max32(const uint32_t (&w)[32]) {
+    float m[11];
+#pragma unroll
+    for (int i = 0; i < 10; ++i)
+        m[i] = max3_nan(__uint_as_float(w[3 * i]), __uint_as_float(w[3 * i + 1]), __uint_as_float(w[3 * i + 2]));
+    m[10] = max_nan(__uint_as_float(w[30]), __uint_as_float(w[31]));
+    float mx = max3_nan(max3_nan(m[0], m[1], m[2]), max3_nan(m[3], m[4], m[5]), max3_nan(m[6], m[7], m[8]));
+    return max3_nan(mx, m[9], m[10]);
 }
 
-bool exp_quantize_supported(long long cols) { return cols > 0 && cols % 32 == 0 && cols <= 262144; }
+// first pass: the block, asking L2 to keep it for the second pass
+__device__ __forceinline__ void load_keep(const float* s, long long b, uint32_t (&w)[32], bool a32) {
+    const char* p = reinterpret_cast<const char*>(s) + b * 128;
+    if (a32) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) ld_v8_keep(p + 32 * i, w + 8 * i);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) ld_2v4(p + 32 * i, w + 8 * i);
+    }
+}
 
+// One row per CTA (TPR threads), CTAs walking
+// rows with a grid stride. Pass 1 streams the row from HBM for its maximum
+// (NaN if any key is NaN), the loads marked to stay in L2; one CTA barrier
+// gives every thread the maximum; pass 2 reads the row again -- from L2 -- and
+// exponentiates and quantizes it block by block. The launcher caps the CTAs
+// in flight so that their rows fit comfortably in L2.
+template <int F, int TPR>
+__global__ void __launch_bounds__(TPR) k_exp_quantize(const float* __restrict__ scores, void* __restrict__ codes,
+                                                     void* __restrict__ scales, long long rows, long long cols,
+                                                     bool a32) {
+    __shared__ float wmax[TPR / 32];
+    __shared__ float rmax;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const long long bpr = cols / 32;
+    const float NEG_INF = __uint_as_float(0xFF800000u);
+    for (long long row = blockIdx.x; row < rows; row += gridDim.x) {
+        const float* s = scores + row * cols;
+        float mx = NEG_INF;
+        long long b = t;
+        for (; b + TPR < bpr; b += 2 * TPR) {  // two blocks in flight
+            uint32_t w0[32], w1[32];
+            load_keep(s, b, w0, a32);
+            load_keep(s, b + TPR, w1, a32);
+            mx = max3_nan(mx, max32(w0), max32(w1));
+        }
+        if (b < bpr) {
+            uint32_t w0[32];
+            load_keep(s, b, w0, a32);
+            mx = max_nan(mx, max32(w0));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = max_nan(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        if constexpr (TPR > 32) {
+            if (lane == 0) wmax[warp] = mx;
+            __syncthreads();
+            if (warp == 0) {
+                float v = lane < TPR / 32 ? wmax[lane] : NEG_INF;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v = max_nan(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+                if (lane == 0) rmax = v;
+            }
+            __syncthreads();
+            mx = rmax;
+        }
+        for (long long bb = t; bb < bpr; bb += TPR) {
+            uint32_t w[32];
+            load_block<float>(s, bb, w, a32);
+            exp_quant_block<F>(w, mx, row * bpr + bb, codes, scales, a32);
+        }
+        if constexpr (TPR > 32) __syncthreads();  // rmax is rewritten for the next row
+    }
+}
+
+bool exp_quantize_supported(long long cols) { return cols > 0 && cols % 32 == 0; }
+
+template <int F, int TPR>
+static cudaError_t launch_xq_t(const float* scores, long long rows, long long cols, void* codes, void* scales,
+                               cudaStream_t st) {
+    auto kern = k_exp_quantize<F, TPR>;
+    int dev = 0, sms = 148, per_sm = 1, l2 = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, TPR, 0);
+    long long ctas = (long long)sms * (per_sm > 0 ? per_sm : 1);
+    // rows in flight x row bytes <= 60% of L2, so pass 2 finds its row there
+    const long long budget = (l2 > 0 ? (long long)l2 : (126LL << 20)) * 3 / 5;
+    const long long by_l2 = budget / (cols * 4);
+    if (by_l2 < ctas) ctas = by_l2 > sms ? by_l2 : sms;
+    if (ctas > rows) ctas = rows;
+    if (ctas < 1) ctas = 1;
+    const bool a32 = ((reinterpret_cast<uintptr_t>(scores) | reinterpret_cast<uintptr_t>(codes)) & 31) == 0;
+    kern<<<(unsigned)ctas, TPR, 0, st>>>(scores, codes, scales, rows, cols, a32);
+    return cudaGetLastError();
+}
+
+// Threads per row: two to four blocks per thread, 32 to 1024 (more, smaller
+// CTAs per SM overlap one row's load phase with another's compute phase).
 template <int F>
 static cudaError_t launch_xq(const float* scores, long long rows, long long cols, void* codes, void* scales,
                              cudaStream_t st) {
     const long long bpr = cols / 32;
-    long long C = (bpr + 127) / 128;  // about 128 blocks (4096 keys) per CTA
-    if (C > 8) C = 8;                 // portable cluster size
-    if (C < 1) C = 1;
-    if ((bpr + C - 1) / C > kMaxThreads) C = 16;  // non-portable size, long rows only
-    const long long per_cta = (bpr + C - 1) / C;
-    const long long nt = (per_cta + 31) / 32 * 32;
-    if (nt > kMaxThreads) return cudaErrorNotSupported;
-    const bool a32 = ((reinterpret_cast<uintptr_t>(scores) | reinterpret_cast<uintptr_t>(codes)) & 31) == 0;
-
-    cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3((unsigned)nt, 1, 1);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (C > 8) {
-        cudaError_t e = cudaFuncSetAttribute(k_exp_quantize<F>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-    }
-    // as many clusters as fit on the GPU at once (each then loops over rows)
-    cfg.gridDim = dim3((unsigned)(C * 1024), 1, 1);
-    int active = 0;
-    if (cudaOccupancyMaxActiveClusters(&active, k_exp_quantize<F>, &cfg) != cudaSuccess || active < 1) {
-        cudaGetLastError();
-        active = 148;
-    }
-    long long G = rows < active ? rows : active;
-    cfg.gridDim = dim3((unsigned)(G * C), 1, 1);
-    return cudaLaunchKernelEx(&cfg, k_exp_quantize<F>, scores, codes, scales, rows, cols, a32);
+    if (bpr <= 64) return launch_xq_t<F, 32>(scores, rows, cols, codes, scales, st);
+    if (bpr <= 128) return launch_xq_t<F, 64>(scores, rows, cols, codes, scales, st);
+    if (bpr <= 256) return launch_xq_t<F, 128>(scores, rows, cols, codes, scales, st);
+    if (bpr <= 1024) return launch_xq_t<F, 256>(scores, rows, cols, codes, scales, st);
+    if (bpr <= 2048) return launch_xq_t<F, 512>(scores, rows, cols, codes, scales, st);
+    return launch_xq_t<F, 1024>(scores, rows, cols, codes, scales, st);
 }
 
 cudaError_t launch_exp_quantize(int fmt, const float* scores, long long rows, long long cols, void* codes,

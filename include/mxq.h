@@ -135,8 +135,7 @@ MXQ_API mxq_status mxq_fake_quantize(mxq_format fmt, const void* src, mxq_dtype 
  *                                         polynomial in fused multiply-adds)
  *   then p is block-quantized exactly like mxq_quantize with dtype MXQ_F32.
  * p is never written to memory. Supported formats: all five (MXFP4 E2M1 is
- * the one the stage feeds). scores 16-byte aligned, cols <= 262144
- * (MXQ_ERR_UNSUPPORTED above that).
+ * the one the stage feeds). scores 16-byte aligned; any cols % 32 == 0.
  */
 MXQ_API mxq_status mxq_exp_quantize(mxq_format fmt, const float* scores, int64_t rows, int64_t cols,
                             void* codes, void* scales, mxq_stream stream);
