@@ -7,8 +7,16 @@ CUDA kernels for NVIDIA B200 (sm_100a) behind a C ABI (include/mxq.h).
     w2 = dequantize(codes, scales, "mxfp6_e2m3", w_bf16.shape)
     g_q = fake_quantize(g_fp32, "axs6")          # quantize + dequantize, one pass
 """
-from .mxq import (EXPORTS, FORMATS, MXQError, dequantize, exp_quantize, fake_quantize, lib, quantize,
-                  quantize_grouped)
+from .mxq import (EXPORTS, FORMATS, MXQError, dequantize, dequantize_cols, exp_quantize, fake_quantize, lib,
+                  quantize, quantize_cols, quantize_grouped)
 
-__all__ = ["quantize", "dequantize", "fake_quantize", "exp_quantize", "quantize_grouped", "MXQError", "FORMATS",
-           "lib", "EXPORTS"]
+
+def fake_quantize_ste(x, fmt="axs6", block_size=32):
+    """Differentiable fake-quantize: forward = fused kernel, backward = identity (STE)."""
+    from .ste import fake_quantize_ste as f
+    return f(x, fmt, block_size)
+
+
+__all__ = ["quantize", "dequantize", "fake_quantize", "fake_quantize_ste", "exp_quantize", "quantize_grouped",
+           "quantize_cols", "dequantize_cols",
+           "MXQError", "FORMATS", "lib", "EXPORTS"]

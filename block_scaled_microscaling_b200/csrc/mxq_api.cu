@@ -159,6 +159,35 @@ mxq_status mxq_exp_quantize(mxq_format fmt, const float* scores, int64_t rows, i
     return from_cuda(mxq::launch_exp_quantize((int)fmt, scores, rows, cols, codes, scales, (cudaStream_t)stream));
 }
 
+mxq_status mxq_quantize_cols(mxq_format fmt, const void* src, mxq_dtype dtype, int64_t rows, int64_t cols,
+                             void* codes, void* scales, mxq_stream stream) {
+    if (!fmt_ok(fmt) || !dtype_ok(dtype)) return MXQ_ERR_INVALID_ARG;
+    if (rows < 0 || rows % 32 != 0 || cols <= 0 || cols % 32 != 0) return MXQ_ERR_SHAPE;
+    if (rows == 0) return MXQ_OK;
+    if (!mxq::cols_grid_ok(rows, cols)) return MXQ_ERR_SHAPE;
+    // same sizes/alignment/overlap rules as the row-direction call on the transpose
+    MXQ_TRY(check_quantize_args(fmt, src, dtype, cols, rows, codes, scales));
+    return from_cuda(mxq::launch_quantize_cols((int)fmt, src, (int)dtype, rows, cols, codes, scales,
+                                               (cudaStream_t)stream));
+}
+
+mxq_status mxq_dequantize_cols(mxq_format fmt, const void* codes, const void* scales, int64_t rows, int64_t cols,
+                               void* dst, mxq_dtype dtype, mxq_stream stream) {
+    if (!fmt_ok(fmt) || !dtype_ok(dtype)) return MXQ_ERR_INVALID_ARG;
+    if (rows < 0 || rows % 32 != 0 || cols <= 0 || cols % 32 != 0) return MXQ_ERR_SHAPE;
+    if (rows == 0) return MXQ_OK;
+    if (!mxq::cols_grid_ok(rows, cols)) return MXQ_ERR_SHAPE;
+    MXQ_TRY(check_shape(cols, rows));
+    MXQ_TRY(check_ptr(codes, 16));
+    MXQ_TRY(check_ptr(scales, scales_align(fmt)));
+    MXQ_TRY(check_ptr(dst, 16));
+    const size_t nd = (size_t)rows * (size_t)cols * dtype_bytes(dtype);
+    if (overlap(dst, nd, codes, codes_bytes(fmt, cols, rows)) || overlap(dst, nd, scales, scales_bytes(fmt, cols, rows)))
+        return MXQ_ERR_INVALID_ARG;
+    return from_cuda(mxq::launch_dequantize_cols((int)fmt, codes, scales, dst, (int)dtype, rows, cols,
+                                                 (cudaStream_t)stream));
+}
+
 size_t mxq_codes_bytes(mxq_format fmt, int64_t rows, int64_t cols) {
     if (!fmt_ok(fmt) || check_shape(rows, cols) != MXQ_OK) return 0;
     return codes_bytes(fmt, rows, cols);

@@ -33,5 +33,11 @@ cudaError_t launch_fake_quantize(int fmt, const void* src, void* dst, int dtype,
 cudaError_t launch_exp_quantize(int fmt, const float* scores, long long rows, long long cols, void* codes,
                                 void* scales, cudaStream_t st);
 bool exp_quantize_supported(long long cols);
+// column-direction blocks (32 rows of a column), transposed output layout
+cudaError_t launch_quantize_cols(int fmt, const void* src, int dtype, long long rows, long long cols, void* codes,
+                                 void* scales, cudaStream_t st);
+cudaError_t launch_dequantize_cols(int fmt, const void* codes, const void* scales, void* dst, int dtype, long long rows,
+                                   long long cols, cudaStream_t st);
+bool cols_grid_ok(long long rows, long long cols);
 
 }  // namespace mxq

@@ -23,7 +23,8 @@ MAX_GROUP = 64
 ELEM_BITS = {"axs6": 6, "mxfp6_e2m3": 6, "mxfp6_e3m2": 6, "mxfp8": 8, "mxfp4": 4}
 
 EXPORTS = ["mxq_quantize", "mxq_dequantize", "mxq_fake_quantize", "mxq_exp_quantize", "mxq_quantize_grouped",
-           "mxq_codes_bytes", "mxq_scales_bytes", "mxq_block_bits", "mxq_status_string", "mxq_version"]
+           "mxq_quantize_cols", "mxq_dequantize_cols", "mxq_codes_bytes", "mxq_scales_bytes", "mxq_block_bits",
+           "mxq_status_string", "mxq_version"]
 
 
 class MXQError(RuntimeError):
@@ -55,6 +56,8 @@ def lib():
             ("mxq_fake_quantize", [i32, vp, i32, i64, i64, vp, vp]),
             ("mxq_exp_quantize", [i32, vp, i64, i64, vp, vp, vp]),
             ("mxq_quantize_grouped", [i32, i32, ctypes.POINTER(_Tensor), i32, vp]),
+            ("mxq_quantize_cols", [i32, vp, i32, i64, i64, vp, vp, vp]),
+            ("mxq_dequantize_cols", [i32, vp, vp, i64, i64, vp, i32, vp]),
         ]:
             fn = getattr(L, name)
             fn.argtypes = args
@@ -97,6 +100,14 @@ def mxq_quantize_grouped(fmt, dtype, tensors, stream):
     for i, (s, c, sc, r, k) in enumerate(tensors):
         arr[i] = _Tensor(s, c, sc, r, k)
     return lib().mxq_quantize_grouped(fmt, dtype, arr, len(tensors), stream)
+
+
+def mxq_quantize_cols(fmt, src, dtype, rows, cols, codes, scales, stream):
+    return lib().mxq_quantize_cols(fmt, src, dtype, rows, cols, codes, scales, stream)
+
+
+def mxq_dequantize_cols(fmt, codes, scales, rows, cols, dst, dtype, stream):
+    return lib().mxq_dequantize_cols(fmt, codes, scales, rows, cols, dst, dtype, stream)
 
 
 def mxq_codes_bytes(fmt, rows, cols):
@@ -250,3 +261,29 @@ def quantize_grouped(xs, fmt, outs=None, stream=None):
         descs.append((x.data_ptr(), c.data_ptr(), s.data_ptr(), r, k))
     _check(mxq_quantize_grouped(_fmt(fmt), dt, descs, _stream(stream)), "mxq_quantize_grouped")
     return outs
+
+
+def quantize_cols(x, fmt, codes=None, scales=None, stream=None):
+    """x [rows, cols] -> blocks of 32 rows per column, laid out as quantize(x.T):
+    codes [cols, rows/32*P], scales [cols, rows/32]."""
+    if not x.is_contiguous() or x.dim() != 2:
+        raise ValueError("x must be a contiguous 2-D tensor")
+    rows, cols = x.shape
+    if codes is None:
+        codes = empty_codes(fmt, cols, rows, x.device)
+    if scales is None:
+        scales = empty_scales(fmt, cols, rows, x.device)
+    _check(mxq_quantize_cols(_fmt(fmt), x.data_ptr(), _dt(x), rows, cols, codes.data_ptr(), scales.data_ptr(),
+                             _stream(stream)), "mxq_quantize_cols")
+    return codes, scales
+
+
+def dequantize_cols(codes, scales, fmt, shape, dtype=None, out=None, stream=None):
+    """Inverse of quantize_cols: values of `shape` = (rows, cols)."""
+    torch = _torch()
+    if out is None:
+        out = torch.empty(tuple(shape), dtype=dtype or torch.bfloat16, device=codes.device)
+    rows, cols = out.shape
+    _check(mxq_dequantize_cols(_fmt(fmt), codes.data_ptr(), scales.data_ptr(), rows, cols, out.data_ptr(), _dt(out),
+                               _stream(stream)), "mxq_dequantize_cols")
+    return out

@@ -159,6 +159,24 @@ typedef struct {
 MXQ_API mxq_status mxq_quantize_grouped(mxq_format fmt, mxq_dtype dtype, const mxq_tensor* tensors, int n,
                                 mxq_stream stream);
 
+/*
+ * Column-direction blocks: each block is 32 consecutive ROWS of one column of
+ * src [rows, cols] (weights stored [in, out]; operands of a backward pass).
+ * The output is exactly what mxq_quantize would produce for the transpose
+ * src^T [cols, rows]: codes [cols, rows/32 * P] and scales [cols, rows/32],
+ * so each column's blocks are contiguous. rows % 32 == 0 and cols % 32 == 0
+ * (MXQ_ERR_SHAPE otherwise), rows <= 16776960. Alignment and overlap rules as
+ * mxq_quantize. ("Sonar: Online MXFP6", Start a model: the blocks of 32 run
+ * along the weight's input dimension.)
+ */
+MXQ_API mxq_status mxq_quantize_cols(mxq_format fmt, const void* src, mxq_dtype dtype, int64_t rows, int64_t cols,
+                                     void* codes, void* scales, mxq_stream stream);
+/* Inverse of mxq_quantize_cols: codes/scales in the transposed layout ->
+ * dst [rows, cols] of type dtype (the values mxq_dequantize gives for the
+ * transpose, transposed back). Same shape rules. */
+MXQ_API mxq_status mxq_dequantize_cols(mxq_format fmt, const void* codes, const void* scales, int64_t rows,
+                                       int64_t cols, void* dst, mxq_dtype dtype, mxq_stream stream);
+
 /* Bytes of the packed code array: rows * cols/32 * payload (0 on bad input). */
 MXQ_API size_t mxq_codes_bytes(mxq_format fmt, int64_t rows, int64_t cols);
 /* Bytes of the scale array: rows * cols/32 (x2 for AXS-6 headers; 0 on bad input). */

@@ -247,3 +247,30 @@ def test_exp_quantize_many_rows_per_cluster(fmt, rows, cols):
     oc, os_ = oracle.exp_quantize(s, fmt)
     assert np.array_equal(host(scales), os_)
     assert np.array_equal(host(codes), oc)
+
+
+# ---- column-direction blocks (32 rows of a column), transposed layout --------------------
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(32, 32), (96, 64), (256, 32), (288, 96), (1024, 160), (4096, 256)])
+def test_quantize_cols_matches_oracle_on_transpose(fmt, dtype, shape):
+    x = hard_values(*shape, dtype, seed=zlib.crc32(repr(("cols", fmt, dtype, shape)).encode()))
+    codes, scales = mxq.quantize_cols(dev(x), fmt)
+    xt = np.ascontiguousarray(x.T)
+    oc, os_ = oracle.quantize(xt, fmt)
+    assert np.array_equal(host(scales), os_)
+    assert np.array_equal(host(codes), oc)
+    out = mxq.dequantize_cols(codes, scales, fmt, shape, tdtype(dtype))
+    ref = oracle.dequantize(oc, os_, fmt, xt.shape, dtype).T
+    assert np.array_equal(bits(host(out)), bits(np.ascontiguousarray(ref)))
+
+
+def test_cols_shape_rules():
+    x = torch.zeros(48, 64, dtype=torch.bfloat16, device="cuda")
+    c = torch.zeros(64 * 48, dtype=torch.uint8, device="cuda")
+    s = torch.zeros(128, dtype=torch.uint8, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream
+    assert mxq.mxq_quantize_cols(1, x.data_ptr(), 1, 48, 64, c.data_ptr(), s.data_ptr(), st) == 2  # rows % 32
+    assert mxq.mxq_quantize_cols(1, x.data_ptr(), 1, 32, 48, c.data_ptr(), s.data_ptr(), st) == 2  # cols % 32
+    assert mxq.mxq_quantize_cols(1, x.data_ptr(), 1, 0, 64, c.data_ptr(), s.data_ptr(), st) == 0   # empty
