@@ -188,6 +188,53 @@ mxq_status mxq_dequantize_cols(mxq_format fmt, const void* codes, const void* sc
                                                  (cudaStream_t)stream));
 }
 
+mxq_status mxq_quantize_exmy(int ebits, int mbits, const void* src, mxq_dtype dtype, int64_t rows, int64_t cols,
+                             void* codes, void* scales, mxq_stream stream) {
+    if (!dtype_ok(dtype)) return MXQ_ERR_INVALID_ARG;
+    if (!mxq::exmy_supported(ebits, mbits)) return MXQ_ERR_UNSUPPORTED;
+    MXQ_TRY(check_shape(rows, cols));
+    if (rows == 0) return MXQ_OK;
+    MXQ_TRY(check_ptr(src, 16));
+    MXQ_TRY(check_ptr(codes, 4));
+    MXQ_TRY(check_ptr(scales, 1));
+    const size_t W = (size_t)(1 + ebits + mbits), nb = (size_t)rows * (size_t)(cols / 32);
+    const size_t nsrc = (size_t)rows * (size_t)cols * dtype_bytes(dtype);
+    if (overlap(src, nsrc, codes, nb * 4 * W) || overlap(src, nsrc, scales, nb) || overlap(codes, nb * 4 * W, scales, nb))
+        return MXQ_ERR_INVALID_ARG;
+    return from_cuda(mxq::launch_exmy(0, ebits, mbits, (int)dtype, src, codes, nullptr, scales, (long long)nb,
+                                      (cudaStream_t)stream));
+}
+
+mxq_status mxq_dequantize_exmy(int ebits, int mbits, const void* codes, const void* scales, int64_t rows, int64_t cols,
+                               void* dst, mxq_dtype dtype, mxq_stream stream) {
+    if (!dtype_ok(dtype)) return MXQ_ERR_INVALID_ARG;
+    if (!mxq::exmy_supported(ebits, mbits)) return MXQ_ERR_UNSUPPORTED;
+    MXQ_TRY(check_shape(rows, cols));
+    if (rows == 0) return MXQ_OK;
+    MXQ_TRY(check_ptr(codes, 4));
+    MXQ_TRY(check_ptr(scales, 1));
+    MXQ_TRY(check_ptr(dst, 16));
+    const size_t W = (size_t)(1 + ebits + mbits), nb = (size_t)rows * (size_t)(cols / 32);
+    const size_t nd = (size_t)rows * (size_t)cols * dtype_bytes(dtype);
+    if (overlap(dst, nd, codes, nb * 4 * W) || overlap(dst, nd, scales, nb)) return MXQ_ERR_INVALID_ARG;
+    return from_cuda(mxq::launch_exmy(1, ebits, mbits, (int)dtype, codes, dst, scales, nullptr, (long long)nb,
+                                      (cudaStream_t)stream));
+}
+
+mxq_status mxq_fake_quantize_exmy(int ebits, int mbits, const void* src, mxq_dtype dtype, int64_t rows, int64_t cols,
+                                  void* dst, mxq_stream stream) {
+    if (!dtype_ok(dtype)) return MXQ_ERR_INVALID_ARG;
+    if (!mxq::exmy_supported(ebits, mbits)) return MXQ_ERR_UNSUPPORTED;
+    MXQ_TRY(check_shape(rows, cols));
+    if (rows == 0) return MXQ_OK;
+    MXQ_TRY(check_ptr(src, 16));
+    MXQ_TRY(check_ptr(dst, 16));
+    const size_t nbytes = (size_t)rows * (size_t)cols * dtype_bytes(dtype);
+    if (src != dst && overlap(src, nbytes, dst, nbytes)) return MXQ_ERR_INVALID_ARG;
+    return from_cuda(mxq::launch_exmy(2, ebits, mbits, (int)dtype, src, dst, nullptr, nullptr,
+                                      (long long)(rows * (cols / 32)), (cudaStream_t)stream));
+}
+
 size_t mxq_codes_bytes(mxq_format fmt, int64_t rows, int64_t cols) {
     if (!fmt_ok(fmt) || check_shape(rows, cols) != MXQ_OK) return 0;
     return codes_bytes(fmt, rows, cols);

@@ -1,0 +1,244 @@
+// mxq_exmy.cu -- generic eXmY element formats (sm_100a).
+//
+// "eXmY: A Data Type and Technique for Arbitrary Bit Precision Quantization",
+// abstract: one data type for any width (3, 5, 6, 7, 9 bits ...) and any
+// split of the bits after the sign into E exponent and M mantissa bits, with
+// dense, byte-addressable packing. Readings (the abstract fixes none): the
+// value of a code is the element-format closed form with bias 2^(E-1) - 1
+// (E >= 1) or 0 (E = 0: sign + fixed-point m / 2^(M-1)); no code is reserved;
+// the block rule is the one of the named formats with emax = 2^(E-1) (0 for
+// E = 0); W = 1 + E + M bit codes are packed LSB-first, so a block's payload is
+// exactly W 32-bit words; the scale is one E8M0 byte.
+//
+// There is no conversion instruction for arbitrary splits, so rounding is
+// integer arithmetic on the fp32 bit pattern of y = |x| * 2^-Es (an exact
+// power-of-two scaling):
+//   normal range   add half an ulp of the target minus one plus the kept
+//                  lsb (round to nearest, ties to even), shift, re-bias;
+//   subnormal      y + 2^(24 - b - M) in fp32 (that binade's ulp is the
+//                  subnormal step) and subtract the constant's bits;
+//   then clamp to the largest magnitude and set the sign bit.
+// Kernels are templated on W (static packing positions) with E, M at run time.
+#include <cstdint>
+#include <cstring>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "mxq_block.cuh"
+#include "mxq_device.cuh"
+#include "mxq_internal.h"
+
+namespace mxq {
+
+constexpr int kExThreads = 256;
+
+struct ExmyParams {
+    int M;            // mantissa bits
+    int emax;         // floor(log2 max)
+    uint32_t maxmag;  // 2^(E+M) - 1
+    uint32_t shift;   // 23 - M
+    uint32_t rebias;  // (127 - b) << M
+    uint32_t sub_lim; // fp32 bits of 2^(1-b): below it the grid step is fixed
+    float sub_c;      // 2^(24 - b - M)
+    float dec_unit;   // 2^(127 - b)
+};
+
+static ExmyParams exmy_params(int E, int M) {
+    const int b = E >= 1 ? (1 << (E - 1)) - 1 : 0;
+    ExmyParams p;
+    p.M = M;
+    p.emax = E >= 1 ? (1 << (E - 1)) : 0;
+    p.maxmag = (1u << (E + M)) - 1u;
+    p.shift = (uint32_t)(23 - M);
+    p.rebias = (uint32_t)(127 - b) << M;
+    p.sub_lim = (uint32_t)(1 - b + 127) << 23;
+    const int ce = 24 - b - M;
+    uint32_t cb = (uint32_t)(ce + 127) << 23;
+    float cf;
+    memcpy(&cf, &cb, 4);
+    p.sub_c = cf;
+    uint32_t db = (uint32_t)(127 - b + 127) << 23;
+    float df;
+    memcpy(&df, &db, 4);
+    p.dec_unit = df;
+    return p;
+}
+
+// magnitude code of y >= 0 (fp32, already scaled)
+__device__ __forceinline__ uint32_t exmy_mag(float y, const ExmyParams& p) {
+    const uint32_t u = __float_as_uint(y);
+    const uint32_t r = u + ((1u << (p.shift - 1)) - 1u) + ((u >> p.shift) & 1u);
+    const uint32_t normal = min((r >> p.shift) - p.rebias, p.maxmag);
+    const uint32_t sub = min(__float_as_uint(y + p.sub_c) - __float_as_uint(p.sub_c), p.maxmag);
+    return u < p.sub_lim ? sub : normal;
+}
+
+template <int W> __device__ __forceinline__ void pack_codes(const uint32_t* c, uint32_t* out) {
+#pragma unroll
+    for (int i = 0; i < W; ++i) out[i] = 0;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        const int bit = W * k, wd = bit >> 5, off = bit & 31;
+        out[wd] |= c[k] << off;
+        if (off + W > 32) out[wd + 1] |= c[k] >> (32 - off);
+    }
+}
+template <int W> __device__ __forceinline__ uint32_t code_of(const uint32_t* pw, int k) {
+    const int bit = W * k, wd = bit >> 5, off = bit & 31;
+    uint32_t c = pw[wd] >> off;
+    if (off + W > 32) c |= pw[wd + 1] << (32 - off);
+    return c & ((1u << W) - 1u);
+}
+
+// values of one block -> W payload words
+template <int W, typename T>
+__device__ __forceinline__ void exmy_encode(const uint32_t* w, uint32_t byte, const ExmyParams& p, uint32_t* out) {
+    const float inv = inv_scale(byte);
+    uint32_t c[32];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        float a, b;
+        upk(f2mul(pair<T>(w, i), dup2(inv)), a, b);
+        c[2 * i] = exmy_mag(fabsf(a), p) | ((__float_as_uint(a) >> 31) << (W - 1));
+        c[2 * i + 1] = exmy_mag(fabsf(b), p) | ((__float_as_uint(b) >> 31) << (W - 1));
+    }
+    pack_codes<W>(c, out);
+    if (byte == 0xFFu) {
+#pragma unroll
+        for (int i = 0; i < W; ++i) out[i] = 0;
+    }
+}
+
+// W payload words -> 32 output values (bf16 pairs or fp32 words)
+template <int W, typename T>
+__device__ __forceinline__ void exmy_decode(const uint32_t* pw, uint32_t byte, const ExmyParams& p, uint32_t* o) {
+    const unsigned long long D = dup2(p.dec_unit), S = dup2(fwd_scale(byte));
+    const uint32_t sh = p.shift;
+    auto bits = [&](uint32_t c) { return ((c & ((1u << (W - 1)) - 1u)) << sh) | ((c >> (W - 1)) << 31); };
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        float a, b;
+        upk(f2mul(f2mul(pk(__uint_as_float(bits(code_of<W>(pw, 2 * i))), __uint_as_float(bits(code_of<W>(pw, 2 * i + 1)))), D), S),
+            a, b);
+        if constexpr (sizeof(T) == 4) {
+            o[2 * i] = __float_as_uint(a);
+            o[2 * i + 1] = __float_as_uint(b);
+        } else {
+            o[i] = bf16x2(a, b);
+        }
+    }
+    if (byte == 0xFFu) {
+#pragma unroll
+        for (int i = 0; i < Blk<T>::NW; ++i) o[i] = sizeof(T) == 4 ? 0x7FC00000u : 0x7FC07FC0u;
+    }
+}
+
+template <int W, typename T>
+__global__ void __launch_bounds__(kExThreads) k_quantize_exmy(const void* __restrict__ src, void* __restrict__ codes,
+                                                              uint8_t* __restrict__ scales, long long nblocks,
+                                                              ExmyParams p, bool a32) {
+    const long long stride = (long long)gridDim.x * kExThreads;
+    for (long long b = (long long)blockIdx.x * kExThreads + threadIdx.x; b < nblocks; b += stride) {
+        uint32_t w[Blk<T>::NW];
+        load_block<T>(src, b, w, a32);
+        const uint32_t am = block_amax<T>(w);
+        const uint32_t byte = am >= 0x7F800000u ? 0xFFu : (uint32_t)max((int)(am >> 23) - p.emax, 0);
+        uint32_t out[W];
+        exmy_encode<W, T>(w, byte, p, out);
+        uint32_t* q = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(codes) + b * 4 * W);
+#pragma unroll
+        for (int i = 0; i < W; ++i) q[i] = out[i];
+        scales[b] = (uint8_t)byte;
+    }
+}
+
+template <int W, typename T>
+__global__ void __launch_bounds__(kExThreads) k_dequantize_exmy(const void* __restrict__ codes,
+                                                                const uint8_t* __restrict__ scales,
+                                                                void* __restrict__ dst, long long nblocks, ExmyParams p,
+                                                                bool a32) {
+    const long long stride = (long long)gridDim.x * kExThreads;
+    for (long long b = (long long)blockIdx.x * kExThreads + threadIdx.x; b < nblocks; b += stride) {
+        uint32_t pw[W];
+        const uint32_t* q = reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(codes) + b * 4 * W);
+#pragma unroll
+        for (int i = 0; i < W; ++i) pw[i] = __ldg(q + i);
+        const uint32_t byte = __ldg(scales + b);
+        uint32_t o[Blk<T>::NW];
+        exmy_decode<W, T>(pw, byte, p, o);
+        store_block<T>(dst, b, o, a32);
+    }
+}
+
+template <int W, typename T>
+__global__ void __launch_bounds__(kExThreads) k_fake_quantize_exmy(const void* src, void* dst, long long nblocks,
+                                                                   ExmyParams p, bool a32) {
+    const long long stride = (long long)gridDim.x * kExThreads;
+    for (long long b = (long long)blockIdx.x * kExThreads + threadIdx.x; b < nblocks; b += stride) {
+        uint32_t w[Blk<T>::NW];
+        load_block<T>(src, b, w, a32);
+        const uint32_t am = block_amax<T>(w);
+        const uint32_t byte = am >= 0x7F800000u ? 0xFFu : (uint32_t)max((int)(am >> 23) - p.emax, 0);
+        uint32_t pw[W], o[Blk<T>::NW];
+        exmy_encode<W, T>(w, byte, p, pw);
+        exmy_decode<W, T>(pw, byte, p, o);
+        store_block<T>(dst, b, o, a32);
+    }
+}
+
+static int ex_grid(const void* fn, long long nb) {
+    int dev = 0, sms = 148, per = 1;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, kExThreads, 0);
+    long long cap = (long long)sms * (per > 0 ? per : 1), want = (nb + kExThreads - 1) / kExThreads;
+    return (int)(want < cap ? (want > 0 ? want : 1) : cap);
+}
+static bool al32(const void* a, const void* b) {
+    return ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b)) & 31) == 0;
+}
+
+template <int W, typename T>
+static cudaError_t ex_launch(int op, const void* in, void* out, const void* aux_in, void* aux_out, long long nb,
+                             const ExmyParams& p, cudaStream_t st) {
+    if (op == 0) {
+        auto k = k_quantize_exmy<W, T>;
+        k<<<ex_grid((const void*)k, nb), kExThreads, 0, st>>>(in, out, reinterpret_cast<uint8_t*>(aux_out), nb, p,
+                                                            al32(in, in));
+    } else if (op == 1) {
+        auto k = k_dequantize_exmy<W, T>;
+        k<<<ex_grid((const void*)k, nb), kExThreads, 0, st>>>(in, reinterpret_cast<const uint8_t*>(aux_in), out, nb, p,
+                                                            al32(out, out));
+    } else {
+        auto k = k_fake_quantize_exmy<W, T>;
+        k<<<ex_grid((const void*)k, nb), kExThreads, 0, st>>>(in, out, nb, p, al32(in, out));
+    }
+    return cudaGetLastError();
+}
+
+bool exmy_supported(int E, int M) { return E >= 0 && E <= 5 && M >= 1 && 1 + E + M >= 3 && 1 + E + M <= 9; }
+
+// op: 0 quantize (in = values, out = codes, aux_out = scales), 1 dequantize
+// (in = codes, aux_in = scales, out = values), 2 fake-quantize (in -> out)
+cudaError_t launch_exmy(int op, int E, int M, int dtype, const void* in, void* out, const void* aux_in, void* aux_out,
+                        long long nb, cudaStream_t st) {
+    if (!exmy_supported(E, M)) return cudaErrorInvalidValue;
+    const ExmyParams p = exmy_params(E, M);
+#define MXQ_EX(WW)                                                                                 \
+    case WW:                                                                                       \
+        return dtype == 1 ? ex_launch<WW, __nv_bfloat16>(op, in, out, aux_in, aux_out, nb, p, st) \
+                          : ex_launch<WW, float>(op, in, out, aux_in, aux_out, nb, p, st);
+    switch (1 + E + M) {
+        MXQ_EX(3)
+        MXQ_EX(4)
+        MXQ_EX(5)
+        MXQ_EX(6)
+        MXQ_EX(7)
+        MXQ_EX(8)
+        MXQ_EX(9)
+    }
+#undef MXQ_EX
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace mxq

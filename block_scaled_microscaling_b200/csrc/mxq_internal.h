@@ -39,5 +39,10 @@ cudaError_t launch_quantize_cols(int fmt, const void* src, int dtype, long long 
 cudaError_t launch_dequantize_cols(int fmt, const void* codes, const void* scales, void* dst, int dtype, long long rows,
                                    long long cols, cudaStream_t st);
 bool cols_grid_ok(long long rows, long long cols);
+// eXmY: op 0 quantize (in values -> out codes, aux_out scales), 1 dequantize
+// (in codes + aux_in scales -> out values), 2 fake-quantize (in -> out)
+bool exmy_supported(int E, int M);
+cudaError_t launch_exmy(int op, int E, int M, int dtype, const void* in, void* out, const void* aux_in, void* aux_out,
+                        long long nblocks, cudaStream_t st);
 
 }  // namespace mxq

@@ -23,8 +23,9 @@ MAX_GROUP = 64
 ELEM_BITS = {"axs6": 6, "mxfp6_e2m3": 6, "mxfp6_e3m2": 6, "mxfp8": 8, "mxfp4": 4}
 
 EXPORTS = ["mxq_quantize", "mxq_dequantize", "mxq_fake_quantize", "mxq_exp_quantize", "mxq_quantize_grouped",
-           "mxq_quantize_cols", "mxq_dequantize_cols", "mxq_codes_bytes", "mxq_scales_bytes", "mxq_block_bits",
-           "mxq_status_string", "mxq_version"]
+           "mxq_quantize_cols", "mxq_dequantize_cols", "mxq_quantize_exmy", "mxq_dequantize_exmy",
+           "mxq_fake_quantize_exmy", "mxq_codes_bytes", "mxq_scales_bytes", "mxq_block_bits", "mxq_status_string",
+           "mxq_version"]
 
 
 class MXQError(RuntimeError):
@@ -58,6 +59,9 @@ def lib():
             ("mxq_quantize_grouped", [i32, i32, ctypes.POINTER(_Tensor), i32, vp]),
             ("mxq_quantize_cols", [i32, vp, i32, i64, i64, vp, vp, vp]),
             ("mxq_dequantize_cols", [i32, vp, vp, i64, i64, vp, i32, vp]),
+            ("mxq_quantize_exmy", [i32, i32, vp, i32, i64, i64, vp, vp, vp]),
+            ("mxq_dequantize_exmy", [i32, i32, vp, vp, i64, i64, vp, i32, vp]),
+            ("mxq_fake_quantize_exmy", [i32, i32, vp, i32, i64, i64, vp, vp]),
         ]:
             fn = getattr(L, name)
             fn.argtypes = args
@@ -108,6 +112,18 @@ def mxq_quantize_cols(fmt, src, dtype, rows, cols, codes, scales, stream):
 
 def mxq_dequantize_cols(fmt, codes, scales, rows, cols, dst, dtype, stream):
     return lib().mxq_dequantize_cols(fmt, codes, scales, rows, cols, dst, dtype, stream)
+
+
+def mxq_quantize_exmy(ebits, mbits, src, dtype, rows, cols, codes, scales, stream):
+    return lib().mxq_quantize_exmy(ebits, mbits, src, dtype, rows, cols, codes, scales, stream)
+
+
+def mxq_dequantize_exmy(ebits, mbits, codes, scales, rows, cols, dst, dtype, stream):
+    return lib().mxq_dequantize_exmy(ebits, mbits, codes, scales, rows, cols, dst, dtype, stream)
+
+
+def mxq_fake_quantize_exmy(ebits, mbits, src, dtype, rows, cols, dst, stream):
+    return lib().mxq_fake_quantize_exmy(ebits, mbits, src, dtype, rows, cols, dst, stream)
 
 
 def mxq_codes_bytes(fmt, rows, cols):
@@ -286,4 +302,42 @@ def dequantize_cols(codes, scales, fmt, shape, dtype=None, out=None, stream=None
     rows, cols = out.shape
     _check(mxq_dequantize_cols(_fmt(fmt), codes.data_ptr(), scales.data_ptr(), rows, cols, out.data_ptr(), _dt(out),
                                _stream(stream)), "mxq_dequantize_cols")
+    return out
+
+
+def quantize_exmy(x, ebits, mbits, codes=None, scales=None, stream=None):
+    """eXmY codes (W = 1 + ebits + mbits bits, W words per block) + E8M0 scales."""
+    torch = _torch()
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    rows, cols = _as2d(x)
+    W = 1 + ebits + mbits
+    if codes is None:
+        codes = torch.empty((rows, (cols // 32) * 4 * W), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((rows, cols // 32), dtype=torch.uint8, device=x.device)
+    _check(mxq_quantize_exmy(ebits, mbits, x.data_ptr(), _dt(x), rows, cols, codes.data_ptr(), scales.data_ptr(),
+                             _stream(stream)), "mxq_quantize_exmy")
+    return codes, scales
+
+
+def dequantize_exmy(codes, scales, ebits, mbits, shape, dtype=None, out=None, stream=None):
+    torch = _torch()
+    if out is None:
+        out = torch.empty(tuple(shape), dtype=dtype or torch.bfloat16, device=codes.device)
+    rows, cols = _as2d(out)
+    _check(mxq_dequantize_exmy(ebits, mbits, codes.data_ptr(), scales.data_ptr(), rows, cols, out.data_ptr(),
+                               _dt(out), _stream(stream)), "mxq_dequantize_exmy")
+    return out
+
+
+def fake_quantize_exmy(x, ebits, mbits, out=None, stream=None):
+    torch = _torch()
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    if out is None:
+        out = torch.empty_like(x)
+    rows, cols = _as2d(x)
+    _check(mxq_fake_quantize_exmy(ebits, mbits, x.data_ptr(), _dt(x), rows, cols, out.data_ptr(), _stream(stream)),
+           "mxq_fake_quantize_exmy")
     return out

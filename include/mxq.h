@@ -177,6 +177,28 @@ MXQ_API mxq_status mxq_quantize_cols(mxq_format fmt, const void* src, mxq_dtype 
 MXQ_API mxq_status mxq_dequantize_cols(mxq_format fmt, const void* codes, const void* scales, int64_t rows,
                                        int64_t cols, void* dst, mxq_dtype dtype, mxq_stream stream);
 
+/*
+ * eXmY element formats ("eXmY" abstract: any bit width, any split of the bits
+ * after the sign into exponent and mantissa, dense byte-addressable packing).
+ * ebits E and mbits M with 0 <= E <= 5, M >= 1, 3 <= W = 1+E+M <= 9
+ * (MXQ_ERR_UNSUPPORTED otherwise). Value of a code: sign, exponent field e,
+ * mantissa m, bias b = 2^(E-1) - 1 (E >= 1) or 0 (E = 0):
+ *   e > 0: 2^(e-b) (1 + m/2^M);  e = 0: 2^(1-b) m/2^M
+ * (E = 0 is sign + fixed point m/2^(M-1)); no code is reserved for Inf/NaN.
+ * Block rule as above with emax = 2^(E-1) (0 for E = 0). Layouts: codes
+ * uint8[rows * cols/32 * 4W] (W-bit codes LSB-first, a block's payload is W
+ * 32-bit words, 4-byte aligned), scales uint8[rows * cols/32] E8M0 bytes.
+ * e2m1 / e2m3 / e3m2 give exactly MXFP4 / MXFP6 E2M3 / E3M2; e0m5 gives AXS-6's
+ * codes (with a one-byte scale). Rounding is integer arithmetic on the fp32
+ * bit patterns (no conversion instruction exists for arbitrary splits).
+ */
+MXQ_API mxq_status mxq_quantize_exmy(int ebits, int mbits, const void* src, mxq_dtype dtype, int64_t rows,
+                                     int64_t cols, void* codes, void* scales, mxq_stream stream);
+MXQ_API mxq_status mxq_dequantize_exmy(int ebits, int mbits, const void* codes, const void* scales, int64_t rows,
+                                       int64_t cols, void* dst, mxq_dtype dtype, mxq_stream stream);
+MXQ_API mxq_status mxq_fake_quantize_exmy(int ebits, int mbits, const void* src, mxq_dtype dtype, int64_t rows,
+                                          int64_t cols, void* dst, mxq_stream stream);
+
 /* Bytes of the packed code array: rows * cols/32 * payload (0 on bad input). */
 MXQ_API size_t mxq_codes_bytes(mxq_format fmt, int64_t rows, int64_t cols);
 /* Bytes of the scale array: rows * cols/32 (x2 for AXS-6 headers; 0 on bad input). */

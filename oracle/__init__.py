@@ -185,3 +185,79 @@ def unpack_codes(codes_block_bytes, fmt):
         for t in range(w):
             out[j] |= np.uint32(bitstr[w * j + t]) << np.uint32(t)
     return out
+
+
+# ---- eXmY formats (E exponent bits, M mantissa bits; see oracle.c) ---------------------
+
+def _exmy_lib():
+    L = lib()
+    if not getattr(L, "_exmy", False):
+        i32, i64, vp = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p
+        L.orc_exmy_decode.restype = ctypes.c_double
+        L.orc_exmy_decode.argtypes = [i32, i32, ctypes.c_uint32]
+        L.orc_exmy_maxval.restype = ctypes.c_double
+        L.orc_exmy_maxval.argtypes = [i32, i32]
+        L.orc_exmy_emax.argtypes = [i32, i32]
+        L.orc_exmy_round_mags.argtypes = [i32, i32, vp, i64, vp]
+        L.orc_quantize_exmy.argtypes = [i32, i32, vp, i32, i64, i64, vp, vp]
+        L.orc_dequantize_exmy.argtypes = [i32, i32, vp, vp, i64, i64, vp, i32]
+        L.orc_fake_quantize_exmy.argtypes = [i32, i32, vp, i32, i64, i64, vp]
+        L._exmy = True
+    return L
+
+
+def exmy_valid(E, M):
+    return 0 <= E <= 5 and M >= 1 and 3 <= 1 + E + M <= 9
+
+
+def exmy_decode_table(E, M):
+    L = _exmy_lib()
+    return np.array([L.orc_exmy_decode(E, M, c) for c in range(1 << (1 + E + M))], dtype=np.float64)
+
+
+def exmy_maxval(E, M):
+    return _exmy_lib().orc_exmy_maxval(E, M)
+
+
+def exmy_emax(E, M):
+    return _exmy_lib().orc_exmy_emax(E, M)
+
+
+def exmy_round_mags(E, M, y):
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    out = np.zeros(y.shape, dtype=np.uint32)
+    _exmy_lib().orc_exmy_round_mags(E, M, _ptr(y), y.size, _ptr(out))
+    return out
+
+
+def quantize_exmy(x, E, M):
+    x = np.ascontiguousarray(x)
+    rows, cols = x.shape
+    W = 1 + E + M
+    codes = np.zeros((rows, cols // 32 * 4 * W), dtype=np.uint8)
+    scales = np.zeros((rows, cols // 32), dtype=np.uint8)
+    rc = _exmy_lib().orc_quantize_exmy(E, M, _ptr(x), DTYPES[_dtype_of(x)], rows, cols, _ptr(codes), _ptr(scales))
+    if rc:
+        raise ValueError(f"oracle quantize_exmy rejected the arguments (rc={rc})")
+    return codes, scales
+
+
+def dequantize_exmy(codes, scales, E, M, shape, dtype="bf16"):
+    rows, cols = shape
+    codes = np.ascontiguousarray(codes)
+    scales = np.ascontiguousarray(scales)
+    out = np.zeros((rows, cols), dtype=np.float32 if dtype == "f32" else np.uint16)
+    rc = _exmy_lib().orc_dequantize_exmy(E, M, _ptr(codes), _ptr(scales), rows, cols, _ptr(out), DTYPES[dtype])
+    if rc:
+        raise ValueError(f"oracle dequantize_exmy rejected the arguments (rc={rc})")
+    return out
+
+
+def fake_quantize_exmy(x, E, M):
+    x = np.ascontiguousarray(x)
+    rows, cols = x.shape
+    out = np.zeros_like(x)
+    rc = _exmy_lib().orc_fake_quantize_exmy(E, M, _ptr(x), DTYPES[_dtype_of(x)], rows, cols, _ptr(out))
+    if rc:
+        raise ValueError(f"oracle fake_quantize_exmy rejected the arguments (rc={rc})")
+    return out

@@ -86,9 +86,7 @@ static uint32_t max_mag(const fmt_t* F) {
 }
 
 /* Value of a code, from the closed forms above. */
-double orc_decode(int f, uint32_t code) {
-    if (!fmt_ok(f)) return NAN;
-    const fmt_t* F = &FMT[f];
+static double decode_f(const fmt_t* F, uint32_t code) {
     uint32_t s = code & sign_mask(F);
     uint32_t mag = code & (sign_mask(F) - 1u);
     double v;
@@ -107,15 +105,16 @@ double orc_decode(int f, uint32_t code) {
     return s ? -v : v;
 }
 
+double orc_decode(int f, uint32_t code) { return fmt_ok(f) ? decode_f(&FMT[f], code) : NAN; }
+
 int orc_bits(int f) { return fmt_ok(f) ? FMT[f].bits : -1; }
 int orc_emax(int f) { return fmt_ok(f) ? FMT[f].emax : -1; }
-double orc_maxval(int f) { return fmt_ok(f) ? orc_decode(f, max_mag(&FMT[f])) : NAN; }
+double orc_maxval(int f) { return fmt_ok(f) ? decode_f(&FMT[f], max_mag(&FMT[f])) : NAN; }
 
 /* Round a finite y >= 0 (already divided by the block scale) to the nearest
  * grid magnitude, ties to the even code, saturating at the largest magnitude. */
-uint32_t orc_round_mag(int f, double y) {
-    const fmt_t* F = &FMT[f];
-    if (y >= orc_maxval(f)) return max_mag(F);
+static uint32_t round_mag_f(const fmt_t* F, double y) {
+    if (y >= decode_f(F, max_mag(F))) return max_mag(F);
     if (F->fixed) return (uint32_t)nearbyint(y * 16.0); /* 16y < 31 here */
     if (y == 0.0) return 0u;
     int e2;
@@ -130,6 +129,8 @@ uint32_t orc_round_mag(int f, double y) {
     if (n < (double)M) return (uint32_t)n;                   /* subnormal: e = 0, m = n  */
     return ((uint32_t)(ey + F->bias) << F->mbits) | ((uint32_t)n - M);
 }
+
+uint32_t orc_round_mag(int f, double y) { return round_mag_f(&FMT[f], y); }
 
 /* orc_round_mag over an array (test harness convenience). */
 void orc_round_mags(int f, const double* y, int64_t n, uint32_t* out) {
@@ -157,8 +158,7 @@ static int block_scale_byte(const fmt_t* F, const double* x, int n) {
 }
 
 /* O1 for one block of 32 values: codes[i] (unpacked) and the scale byte. */
-int orc_quantize_block(int f, const double* x, uint32_t* codes) {
-    const fmt_t* F = &FMT[f];
+static int quantize_block_f(const fmt_t* F, const double* x, uint32_t* codes) {
     int byte = block_scale_byte(F, x, 32);
     if (byte == 0xFF) {
         for (int i = 0; i < 32; ++i) codes[i] = 0u;
@@ -167,11 +167,13 @@ int orc_quantize_block(int f, const double* x, uint32_t* codes) {
     int Es = byte - 127;
     for (int i = 0; i < 32; ++i) {
         double y = ldexp(fabs(x[i]), -Es);            /* exact power-of-two scaling */
-        uint32_t mag = orc_round_mag(f, y);
+        uint32_t mag = round_mag_f(F, y);
         codes[i] = (signbit(x[i]) ? sign_mask(F) : 0u) | mag;
     }
     return byte;
 }
+
+int orc_quantize_block(int f, const double* x, uint32_t* codes) { return quantize_block_f(&FMT[f], x, codes); }
 
 /* ---- value types ------------------------------------------------------- */
 
@@ -285,20 +287,47 @@ static int check(int f, int dtype, int64_t rows, int64_t cols) {
     return 0;
 }
 
-int orc_quantize(int f, const void* src, int dtype, int64_t rows, int64_t cols,
-                 uint8_t* codes, void* scales) {
-    int rc = check(f, dtype, rows, cols);
-    if (rc) return rc;
-    const fmt_t* F = &FMT[f];
-    int64_t nb = rows * (cols / 32);
+static void quantize_f(const fmt_t* F, const void* src, int dtype, int64_t nb, uint8_t* codes, void* scales) {
     double x[32];
     uint32_t c[32];
     for (int64_t b = 0; b < nb; ++b) {
         for (int i = 0; i < 32; ++i) x[i] = load_value(src, dtype, 32 * b + i);
-        int byte = orc_quantize_block(f, x, c);
+        int byte = quantize_block_f(F, x, c);
         pack_block(F, c, codes + b * payload_bytes(F));
         store_scale(F, scales, b, byte);
     }
+}
+
+static void dequantize_f(const fmt_t* F, const uint8_t* codes, const void* scales, int64_t nb, void* dst, int dtype) {
+    uint32_t c[32];
+    for (int64_t b = 0; b < nb; ++b) {
+        unpack_block(F, codes + b * payload_bytes(F), c);
+        int byte = load_scale(F, scales, b);
+        for (int i = 0; i < 32; ++i) {
+            double v = (byte == 0xFF) ? NAN : ldexp(decode_f(F, c[i]), byte - 127);
+            store_value(dst, dtype, 32 * b + i, v);
+        }
+    }
+}
+
+static void fake_quantize_f(const fmt_t* F, const void* src, int dtype, int64_t nb, void* dst) {
+    double x[32];
+    uint32_t c[32];
+    for (int64_t b = 0; b < nb; ++b) {
+        for (int i = 0; i < 32; ++i) x[i] = load_value(src, dtype, 32 * b + i);
+        int byte = quantize_block_f(F, x, c);
+        for (int i = 0; i < 32; ++i) {
+            double v = (byte == 0xFF) ? NAN : ldexp(decode_f(F, c[i]), byte - 127);
+            store_value(dst, dtype, 32 * b + i, v);
+        }
+    }
+}
+
+int orc_quantize(int f, const void* src, int dtype, int64_t rows, int64_t cols,
+                 uint8_t* codes, void* scales) {
+    int rc = check(f, dtype, rows, cols);
+    if (rc) return rc;
+    quantize_f(&FMT[f], src, dtype, rows * (cols / 32), codes, scales);
     return 0;
 }
 
@@ -306,34 +335,90 @@ int orc_dequantize(int f, const uint8_t* codes, const void* scales, int64_t rows
                    void* dst, int dtype) {
     int rc = check(f, dtype, rows, cols);
     if (rc) return rc;
-    const fmt_t* F = &FMT[f];
-    int64_t nb = rows * (cols / 32);
-    uint32_t c[32];
-    for (int64_t b = 0; b < nb; ++b) {
-        unpack_block(F, codes + b * payload_bytes(F), c);
-        int byte = load_scale(F, scales, b);
-        for (int i = 0; i < 32; ++i) {
-            double v = (byte == 0xFF) ? NAN : ldexp(orc_decode(f, c[i]), byte - 127);
-            store_value(dst, dtype, 32 * b + i, v);
-        }
-    }
+    dequantize_f(&FMT[f], codes, scales, rows * (cols / 32), dst, dtype);
     return 0;
 }
 
 int orc_fake_quantize(int f, const void* src, int dtype, int64_t rows, int64_t cols, void* dst) {
     int rc = check(f, dtype, rows, cols);
     if (rc) return rc;
-    int64_t nb = rows * (cols / 32);
-    double x[32];
-    uint32_t c[32];
-    for (int64_t b = 0; b < nb; ++b) {
-        for (int i = 0; i < 32; ++i) x[i] = load_value(src, dtype, 32 * b + i);
-        int byte = orc_quantize_block(f, x, c);
-        for (int i = 0; i < 32; ++i) {
-            double v = (byte == 0xFF) ? NAN : ldexp(orc_decode(f, c[i]), byte - 127);
-            store_value(dst, dtype, 32 * b + i, v);
-        }
-    }
+    fake_quantize_f(&FMT[f], src, dtype, rows * (cols / 32), dst);
+    return 0;
+}
+
+/* ---- eXmY element formats ---------------------------------------------- */
+/*
+ * [EXMY] abstract: a data type for any bit width (3, 5, 6, 7, 9 bits ...) and
+ * every split of the bits after the sign into exponent and mantissa (e.g.
+ * e0m6 ... e6m0 at 7 bits), with dense byte-addressable packing.
+ * Readings (the abstract fixes none of them): value of a code with E exponent
+ * bits and M mantissa bits as in the element formats above, with bias
+ * b = 2^(E-1) - 1 for E >= 1 and b = 0 for E = 0 (a sign + fixed-point
+ * magnitude m / 2^(M-1)); no code is reserved for Inf or NaN; the shared scale
+ * and rounding rules are the block rule above with emax = 2^(E-1) (0 when
+ * E = 0); codes packed LSB-first, W = 1 + E + M bits each, so a block's payload
+ * is 4W bytes; the scale is one E8M0 byte. Supported: 0 <= E <= 5, M >= 1,
+ * 3 <= W <= 9. (e2m1, e2m3 and e3m2 are then MXFP4 / MXFP6; e0m5 is AXS-6.)
+ */
+static int exmy_desc(int E, int M, fmt_t* F) {
+    if (E < 0 || E > 5 || M < 1 || 1 + E + M < 3 || 1 + E + M > 9) return 1;
+    F->bits = 1 + E + M;
+    F->mbits = M;
+    F->bias = E >= 1 ? (1 << (E - 1)) - 1 : 0;
+    F->emax = E >= 1 ? (1 << (E - 1)) : 0;
+    F->fixed = 0;
+    F->nan_mag = -1;
+    return 0;
+}
+
+double orc_exmy_decode(int E, int M, uint32_t code) {
+    fmt_t F;
+    return exmy_desc(E, M, &F) ? NAN : decode_f(&F, code);
+}
+
+double orc_exmy_maxval(int E, int M) {
+    fmt_t F;
+    return exmy_desc(E, M, &F) ? NAN : decode_f(&F, max_mag(&F));
+}
+
+int orc_exmy_emax(int E, int M) {
+    fmt_t F;
+    return exmy_desc(E, M, &F) ? -1 : F.emax;
+}
+
+void orc_exmy_round_mags(int E, int M, const double* y, int64_t n, uint32_t* out) {
+    fmt_t F;
+    if (exmy_desc(E, M, &F)) return;
+    for (int64_t i = 0; i < n; ++i) out[i] = round_mag_f(&F, y[i]);
+}
+
+int orc_quantize_exmy(int E, int M, const void* src, int dtype, int64_t rows, int64_t cols,
+                      uint8_t* codes, uint8_t* scales) {
+    fmt_t F;
+    if (exmy_desc(E, M, &F)) return 1;
+    int rc = check(0, dtype, rows, cols);
+    if (rc) return rc;
+    quantize_f(&F, src, dtype, rows * (cols / 32), codes, scales);
+    return 0;
+}
+
+int orc_dequantize_exmy(int E, int M, const uint8_t* codes, const uint8_t* scales, int64_t rows,
+                        int64_t cols, void* dst, int dtype) {
+    fmt_t F;
+    if (exmy_desc(E, M, &F)) return 1;
+    int rc = check(0, dtype, rows, cols);
+    if (rc) return rc;
+    dequantize_f(&F, codes, scales, rows * (cols / 32), dst, dtype);
+    return 0;
+}
+
+int orc_fake_quantize_exmy(int E, int M, const void* src, int dtype, int64_t rows, int64_t cols,
+                           void* dst) {
+    fmt_t F;
+    if (exmy_desc(E, M, &F)) return 1;
+    int rc = check(0, dtype, rows, cols);
+    if (rc) return rc;
+    fake_quantize_f(&F, src, dtype, rows * (cols / 32), dst);
     return 0;
 }
 

@@ -1,0 +1,58 @@
+"""GPU parity for the eXmY formats (integer rounding path) against the oracle, bit for bit."""
+import numpy as np
+import pytest
+
+import oracle
+
+torch = pytest.importorskip("torch")
+from block_scaled_microscaling_b200 import mxq  # noqa: E402
+
+from test_parity_gpu import bits, dev, hard_values, host, tdtype  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+SPLITS = [(E, M) for W in range(3, 10) for E in range(0, 6) for M in [W - 1 - E] if oracle.exmy_valid(E, M)]
+
+
+@pytest.mark.parametrize("E,M", SPLITS)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_quantize_and_fake_quantize_match_oracle(E, M, dtype):
+    x = hard_values(67, 160, dtype, seed=100 * E + M)
+    codes, scales = mxq.quantize_exmy(dev(x), E, M)
+    oc, os_ = oracle.quantize_exmy(x, E, M)
+    assert np.array_equal(host(scales), os_)
+    assert np.array_equal(host(codes), oc)
+    fq = mxq.fake_quantize_exmy(dev(x), E, M)
+    assert np.array_equal(bits(host(fq)), bits(oracle.fake_quantize_exmy(x, E, M)))
+
+
+@pytest.mark.parametrize("E,M", SPLITS)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_dequantize_random_codes_match_oracle(E, M, dtype):
+    rows, cols = 40, 256
+    W = 1 + E + M
+    rng = np.random.default_rng(7 * E + M)
+    codes = rng.integers(0, 256, (rows, cols // 32 * 4 * W), dtype=np.uint8)
+    scales = rng.integers(0, 256, (rows, cols // 32), dtype=np.uint8)
+    scales.reshape(-1)[:256] = np.arange(256)
+    out = mxq.dequantize_exmy(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(), E, M, (rows, cols),
+                              tdtype(dtype))
+    ref = oracle.dequantize_exmy(codes, scales, E, M, (rows, cols), dtype)
+    assert np.array_equal(bits(host(out)), bits(ref))
+
+
+@pytest.mark.parametrize("E,M,fmt", [(2, 1, "mxfp4"), (2, 3, "mxfp6_e2m3"), (3, 2, "mxfp6_e3m2")])
+def test_named_splits_agree_with_the_conversion_instruction_path(E, M, fmt):
+    x = hard_values(129, 256, "bf16", seed=3)
+    c1, s1 = mxq.quantize_exmy(dev(x), E, M)
+    c2, s2 = mxq.quantize(dev(x), fmt)
+    assert torch.equal(c1, c2) and torch.equal(s1, s2)
+
+
+def test_unsupported_split():
+    x = torch.zeros(1, 32, device="cuda")
+    c = torch.zeros(64, dtype=torch.uint8, device="cuda")
+    s = torch.zeros(1, dtype=torch.uint8, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream
+    assert mxq.mxq_quantize_exmy(6, 2, x.data_ptr(), 0, 1, 32, c.data_ptr(), s.data_ptr(), st) == 4
+    assert mxq.mxq_quantize_exmy(1, 8, x.data_ptr(), 0, 1, 32, c.data_ptr(), s.data_ptr(), st) == 4
