@@ -387,8 +387,8 @@ def workloads_breakdown(torch, mxq, hbm):
     return out
 
 
-PROFILE_CASES = ["q_e2m3_weight", "dq_e2m3_weight", "q_mxfp8_act", "dq_mxfp8_act", "q_axs6_layer",
-                 "q_e2m3_layer", "fq_axs6_grad", "exp_mxfp4_scores"]
+PROFILE_CASES = ["q_e2m3_weight", "q_e3m2_weight", "dq_e2m3_weight", "q_mxfp8_act", "dq_mxfp8_act", "q_axs6_layer",
+                 "q_e2m3_layer", "fq_axs6_grad", "exp_mxfp4_scores", "qcols_e2m3_weight", "exmy_e3m3_act"]
 
 
 def profile_case(name, reps):
@@ -397,13 +397,22 @@ def profile_case(name, reps):
     from block_scaled_microscaling_b200 import mxq
     dev = torch.device("cuda")
     gen = torch.Generator(device=dev).manual_seed(0)
-    if name in ("q_e2m3_weight", "dq_e2m3_weight"):
+    if name in ("q_e2m3_weight", "q_e3m2_weight", "dq_e2m3_weight", "qcols_e2m3_weight"):
         w_host, _ = synthetic.weight_with_outliers(seed=1)
         x = torch.from_numpy(w_host.view(np.int16)).view(torch.bfloat16).cuda()
-        c, s = mxq.quantize(x, "mxfp6_e2m3")
+        f = "mxfp6_e3m2" if "e3m2" in name else "mxfp6_e2m3"
+        c, s = mxq.quantize(x, f)
         y = torch.empty_like(x)
-        fn = (lambda: mxq.quantize(x, "mxfp6_e2m3", codes=c, scales=s)) if name[0] == "q" else \
-            (lambda: mxq.dequantize(c, s, "mxfp6_e2m3", x.shape, out=y))
+        if name.startswith("qcols"):
+            fn = lambda: mxq.quantize_cols(x, f, codes=c, scales=s)
+        elif name[0] == "q":
+            fn = lambda: mxq.quantize(x, f, codes=c, scales=s)
+        else:
+            fn = lambda: mxq.dequantize(c, s, f, x.shape, out=y)
+    elif name == "exmy_e3m3_act":
+        x = (torch.randn(16384, 8192, device=dev, generator=gen) * 0.5).to(torch.bfloat16)
+        c, s = mxq.quantize_exmy(x, 3, 3)
+        fn = lambda: mxq.quantize_exmy(x, 3, 3, codes=c, scales=s)
     elif name in ("q_mxfp8_act", "dq_mxfp8_act"):
         x = (torch.randn(16384, 8192, device=dev, generator=gen) * 0.5).to(torch.bfloat16)
         c, s = mxq.quantize(x, "mxfp8")
