@@ -261,3 +261,36 @@ def fake_quantize_exmy(x, E, M):
     if rc:
         raise ValueError(f"oracle fake_quantize_exmy rejected the arguments (rc={rc})")
     return out
+
+
+# ---- scale-factor layout of the block-scaled MMA (see oracle.c) -------------------------
+
+def _mma_lib():
+    L = lib()
+    if not getattr(L, "_mma", False):
+        i64, vp = ctypes.c_int64, ctypes.c_void_p
+        L.orc_mma_scales_bytes.restype = i64
+        L.orc_mma_scales_bytes.argtypes = [i64, i64]
+        L.orc_mma_scale_index.restype = i64
+        L.orc_mma_scale_index.argtypes = [i64, i64, i64]
+        L.orc_swizzle_scales.argtypes = [vp, i64, i64, vp]
+        L._mma = True
+    return L
+
+
+def mma_scales_bytes(rows, kb):
+    return _mma_lib().orc_mma_scales_bytes(rows, kb)
+
+
+def mma_scale_index(r, k, kb):
+    return _mma_lib().orc_mma_scale_index(r, k, kb)
+
+
+def swizzle_scales(scales):
+    """[rows, kb] uint8 E8M0 scales -> 1-D uint8 array in the block-scaled MMA layout."""
+    s = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, kb = s.shape
+    out = np.zeros(mma_scales_bytes(rows, kb), dtype=np.uint8)
+    if _mma_lib().orc_swizzle_scales(_ptr(s), rows, kb, _ptr(out)):
+        raise ValueError("oracle swizzle_scales rejected the arguments")
+    return out

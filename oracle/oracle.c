@@ -509,3 +509,41 @@ int64_t orc_codes_bytes(int f, int64_t rows, int64_t cols) {
 int64_t orc_scales_bytes(int f, int64_t rows, int64_t cols) {
     return fmt_ok(f) ? rows * (cols / 32) * (FMT[f].fixed ? 2 : 1) : -1;
 }
+
+/*
+ * Scale-factor layout read by the block-scaled tensor-core MMA.
+ *
+ * The pages do not define it: "Sonar: Online MXFP6" (Current limits) runs its
+ * converted weights through block-scaled GEMM kernels with dense dimensions in
+ * multiples of 128, and those kernels read the per-block E8M0 scales in the
+ * layout of the hardware's block-scaled MMA (NVIDIA cuBLAS documentation,
+ * "1D block scaling factors layout"). Reading adopted, written out from that
+ * definition:
+ *   - the [rows, kb] scale matrix (kb = blocks of 32 along K per row) is
+ *     padded with zero bytes to rows128 = ceil(rows/128)*128 rows and
+ *     kb4 = ceil(kb/4)*4 columns;
+ *   - it is cut into tiles of 128 rows x 4 columns, 512 bytes each, stored
+ *     tile-row by tile-row: tile (R, C) starts at byte (R * kb4/4 + C) * 512;
+ *   - inside a tile, row r (0..127) and column c (0..3) sit at byte
+ *     (r % 32) * 16 + (r / 32) * 4 + c.
+ */
+int64_t orc_mma_scales_bytes(int64_t rows, int64_t kb) {
+    if (rows < 0 || kb < 0) return -1;
+    return ((rows + 127) / 128) * 128 * (((kb + 3) / 4) * 4);
+}
+
+int64_t orc_mma_scale_index(int64_t r, int64_t k, int64_t kb) {
+    const int64_t tiles_per_row = (kb + 3) / 4;
+    const int64_t tile = (r / 128) * tiles_per_row + k / 4;
+    const int64_t rr = r % 128;
+    return tile * 512 + (rr % 32) * 16 + (rr / 32) * 4 + (k % 4);
+}
+
+int orc_swizzle_scales(const uint8_t* scales, int64_t rows, int64_t kb, uint8_t* out) {
+    if (rows < 0 || kb <= 0) return 1;
+    const int64_t n = orc_mma_scales_bytes(rows, kb);
+    for (int64_t i = 0; i < n; ++i) out[i] = 0;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < kb; ++k) out[orc_mma_scale_index(r, k, kb)] = scales[r * kb + k];
+    return 0;
+}
