@@ -106,6 +106,46 @@ mxq_status mxq_quantize(mxq_format fmt, const void* src, mxq_dtype dtype, int64_
     return from_cuda(mxq::launch_quantize<1>((int)fmt, (int)dtype, tab, (cudaStream_t)stream));
 }
 
+size_t mxq_mma_scales_bytes(int64_t rows, int64_t cols) {
+    if (check_shape(rows, cols) != MXQ_OK) return 0;
+    return (size_t)((rows + 127) / 128) * 128 * (size_t)(((cols / 32) + 3) / 4) * 4;
+}
+
+mxq_status mxq_quantize_mma(mxq_format fmt, const void* src, mxq_dtype dtype, int64_t rows, int64_t cols,
+                            void* codes, void* scales, mxq_stream stream) {
+    if (!fmt_ok(fmt) || !dtype_ok(dtype)) return MXQ_ERR_INVALID_ARG;
+    if (fmt == MXQ_AXS6) return MXQ_ERR_UNSUPPORTED;
+    MXQ_TRY(check_shape(rows, cols));
+    if (rows == 0) return MXQ_OK;
+    MXQ_TRY(check_ptr(src, 16));
+    MXQ_TRY(check_ptr(codes, 16));
+    MXQ_TRY(check_ptr(scales, 1));
+    const size_t nsrc = (size_t)rows * (size_t)cols * dtype_bytes(dtype);
+    const size_t nc = codes_bytes(fmt, rows, cols), ns = mxq_mma_scales_bytes(rows, cols);
+    if (overlap(src, nsrc, codes, nc) || overlap(src, nsrc, scales, ns) || overlap(codes, nc, scales, ns))
+        return MXQ_ERR_INVALID_ARG;
+    const int64_t kb = cols / 32;
+    if (rows % 128 != 0 || kb % 4 != 0) {
+        cudaError_t e = cudaMemsetAsync(scales, 0, ns, (cudaStream_t)stream);
+        if (e != cudaSuccess) return from_cuda(e);
+    }
+    mxq::SegTable<1> tab{};
+    tab.seg[0] = {src, codes, scales, rows * kb, 0, kb};
+    tab.n = 1;
+    return from_cuda(mxq::launch_quantize<1>((int)fmt, (int)dtype, tab, (cudaStream_t)stream));
+}
+
+mxq_status mxq_swizzle_scales(const void* scales, int64_t rows, int64_t kblocks, void* out, mxq_stream stream) {
+    if (rows < 0 || kblocks <= 0 || kblocks > kMaxElems / 32) return MXQ_ERR_SHAPE;
+    MXQ_TRY(check_shape(rows, 32 * kblocks));
+    if (rows == 0) return MXQ_OK;
+    MXQ_TRY(check_ptr(scales, 1));
+    MXQ_TRY(check_ptr(out, 4));
+    if (overlap(scales, (size_t)rows * (size_t)kblocks, out, mxq_mma_scales_bytes(rows, 32 * kblocks)))
+        return MXQ_ERR_INVALID_ARG;
+    return from_cuda(mxq::launch_swizzle_scales(scales, rows, kblocks, out, (cudaStream_t)stream));
+}
+
 mxq_status mxq_quantize_grouped(mxq_format fmt, mxq_dtype dtype, const mxq_tensor* tensors, int n,
                                 mxq_stream stream) {
     if (!fmt_ok(fmt) || !dtype_ok(dtype) || tensors == nullptr || n < 1 || n > MXQ_MAX_GROUP)

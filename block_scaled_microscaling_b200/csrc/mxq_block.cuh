@@ -152,6 +152,24 @@ __device__ __forceinline__ void store_scale(void* scales, long long b, uint32_t 
     if constexpr (Fmt<F>::FIXED) reinterpret_cast<uint16_t*>(scales)[b] = (uint16_t)byte;  // config = 0
     else reinterpret_cast<uint8_t*>(scales)[b] = (uint8_t)byte;
 }
+// Byte offset of block b's scale (b = r * kb + k, kb blocks per row) in the
+// scale layout of the block-scaled tensor-core MMA: [rows, kb] padded to
+// multiples of 128 x 4, cut into 128 x 4 tiles of 512 bytes stored tile-row by
+// tile-row, row r / column c of a tile at byte (r % 32) * 16 + (r / 32) * 4 + c.
+__device__ __forceinline__ long long mma_scale_offset(long long b, long long kb) {
+    long long r, k;
+    if ((unsigned long long)b <= 0xFFFFFFFFull && (unsigned long long)kb <= 0xFFFFFFFFull) {
+        const uint32_t r32 = (uint32_t)b / (uint32_t)kb;
+        r = r32;
+        k = (long long)((uint32_t)b - r32 * (uint32_t)kb);
+    } else {
+        r = b / kb;
+        k = b - r * kb;
+    }
+    const long long tiles = (kb + 3) >> 2;
+    return ((((r >> 7) * tiles) + (k >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (k & 3);
+}
+
 template <int F>
 __device__ __forceinline__ uint32_t load_scale(const void* scales, long long b) {
     if constexpr (Fmt<F>::FIXED) return __ldg(reinterpret_cast<const uint16_t*>(scales) + b) & 0xFFu;

@@ -75,8 +75,11 @@ __device__ __forceinline__ void warp_store6(void* codes, long long first_blk, in
     __syncwarp();
 }
 
-template <int F, typename T, int NSEG>
+// MMA: scales go to the block-scaled MMA tile layout (single tensor, E8M0 formats); a separate
+// instantiation, so the plain and grouped kernels carry no trace of it.
+template <int F, typename T, int NSEG, bool MMA = false>
 __global__ void __launch_bounds__(kThreads) k_quantize(const __grid_constant__ SegTable<NSEG> tab) {
+    static_assert(!MMA || (NSEG == 1 && !Fmt<F>::FIXED), "tile-layout scales: one tensor, E8M0 format");
     constexpr int U = q_unroll<F, T, NSEG>();
     constexpr bool STAGE = q_stage<F, T, NSEG>();
     __shared__ __align__(16) uint8_t stage[STAGE ? kThreads / 32 : 1][STAGE ? 32 * 24 : 16];
@@ -117,7 +120,12 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const __grid_constant__ S
             } else {
                 if (ok[u]) store_payload<F>(g[u]->codes, b[u], out, a32[u]);
             }
-            if (ok[u]) store_scale<F>(g[u]->scales, b[u], byte);
+            if (ok[u]) {
+                if constexpr (MMA)
+                    reinterpret_cast<uint8_t*>(g[u]->scales)[mma_scale_offset(b[u], g[u]->kb_mma)] = (uint8_t)byte;
+                else
+                    store_scale<F>(g[u]->scales, b[u], byte);
+            }
         }
     }
 }
@@ -209,6 +217,11 @@ static bool aligned32(const void* a, const void* b) {
 template <int F, typename T, int NSEG>
 static cudaError_t launch_q(const SegTable<NSEG>& tab, cudaStream_t st) {
     auto k = k_quantize<F, T, NSEG>;
+    if constexpr (NSEG == 1 && !Fmt<F>::FIXED) {
+        if (tab.seg[0].kb_mma) k = k_quantize<F, T, 1, true>;
+    } else {
+        if (tab.seg[0].kb_mma) return cudaErrorInvalidValue;
+    }
     k<<<grid_for(k, tab.nblocks), kThreads, 0, st>>>(tab);
     return cudaGetLastError();
 }

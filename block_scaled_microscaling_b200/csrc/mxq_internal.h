@@ -15,6 +15,7 @@ struct Seg {
     void* scales;
     long long nblocks;  // blocks of 32 values
     long long blk0;     // first block of this tensor in the concatenation (filled by the launcher)
+    long long kb_mma;   // 0: scales [rows, cols/32] row-major; else blocks per row, scales in the MMA tile layout
 };
 template <int N> struct SegTable {
     Seg seg[N];
@@ -39,6 +40,8 @@ cudaError_t launch_quantize_cols(int fmt, const void* src, int dtype, long long 
 cudaError_t launch_dequantize_cols(int fmt, const void* codes, const void* scales, void* dst, int dtype, long long rows,
                                    long long cols, cudaStream_t st);
 bool cols_grid_ok(long long rows, long long cols);
+// plain [rows, kb] E8M0 scales -> block-scaled MMA tile layout (padding written as 0)
+cudaError_t launch_swizzle_scales(const void* scales, long long rows, long long kb, void* out, cudaStream_t st);
 // eXmY: op 0 quantize (in values -> out codes, aux_out scales), 1 dequantize
 // (in codes + aux_in scales -> out values), 2 fake-quantize (in -> out)
 bool exmy_supported(int E, int M);

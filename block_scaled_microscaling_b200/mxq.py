@@ -24,7 +24,8 @@ ELEM_BITS = {"axs6": 6, "mxfp6_e2m3": 6, "mxfp6_e3m2": 6, "mxfp8": 8, "mxfp4": 4
 
 EXPORTS = ["mxq_quantize", "mxq_dequantize", "mxq_fake_quantize", "mxq_exp_quantize", "mxq_quantize_grouped",
            "mxq_quantize_cols", "mxq_dequantize_cols", "mxq_quantize_exmy", "mxq_dequantize_exmy",
-           "mxq_fake_quantize_exmy", "mxq_codes_bytes", "mxq_scales_bytes", "mxq_block_bits", "mxq_status_string",
+           "mxq_fake_quantize_exmy", "mxq_quantize_mma", "mxq_swizzle_scales", "mxq_mma_scales_bytes",
+           "mxq_codes_bytes", "mxq_scales_bytes", "mxq_block_bits", "mxq_status_string",
            "mxq_version"]
 
 
@@ -62,6 +63,8 @@ def lib():
             ("mxq_quantize_exmy", [i32, i32, vp, i32, i64, i64, vp, vp, vp]),
             ("mxq_dequantize_exmy", [i32, i32, vp, vp, i64, i64, vp, i32, vp]),
             ("mxq_fake_quantize_exmy", [i32, i32, vp, i32, i64, i64, vp, vp]),
+            ("mxq_quantize_mma", [i32, vp, i32, i64, i64, vp, vp, vp]),
+            ("mxq_swizzle_scales", [vp, i64, i64, vp, vp]),
         ]:
             fn = getattr(L, name)
             fn.argtypes = args
@@ -70,6 +73,8 @@ def lib():
         L.mxq_codes_bytes.restype = sz
         L.mxq_scales_bytes.argtypes = [i32, i64, i64]
         L.mxq_scales_bytes.restype = sz
+        L.mxq_mma_scales_bytes.argtypes = [i64, i64]
+        L.mxq_mma_scales_bytes.restype = sz
         L.mxq_block_bits.argtypes = [i32]
         L.mxq_block_bits.restype = i32
         L.mxq_status_string.argtypes = [i32]
@@ -124,6 +129,18 @@ def mxq_dequantize_exmy(ebits, mbits, codes, scales, rows, cols, dst, dtype, str
 
 def mxq_fake_quantize_exmy(ebits, mbits, src, dtype, rows, cols, dst, stream):
     return lib().mxq_fake_quantize_exmy(ebits, mbits, src, dtype, rows, cols, dst, stream)
+
+
+def mxq_quantize_mma(fmt, src, dtype, rows, cols, codes, scales, stream):
+    return lib().mxq_quantize_mma(fmt, src, dtype, rows, cols, codes, scales, stream)
+
+
+def mxq_swizzle_scales(scales, rows, kblocks, out, stream):
+    return lib().mxq_swizzle_scales(scales, rows, kblocks, out, stream)
+
+
+def mxq_mma_scales_bytes(rows, cols):
+    return lib().mxq_mma_scales_bytes(rows, cols)
 
 
 def mxq_codes_bytes(fmt, rows, cols):
@@ -255,6 +272,34 @@ def exp_quantize(scores, fmt="mxfp4", codes=None, scales=None, stream=None):
     _check(mxq_exp_quantize(_fmt(fmt), scores.data_ptr(), rows, cols, codes.data_ptr(), scales.data_ptr(),
                             _stream(stream)), "mxq_exp_quantize")
     return codes, scales
+
+
+def quantize_mma(x, fmt, codes=None, scales=None, stream=None):
+    """As quantize, with the scales as a 1-D uint8 tensor in the block-scaled MMA tile layout
+    (mxq_mma_scales_bytes(rows, cols) bytes, zero padding)."""
+    torch = _torch()
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    rows, cols = _as2d(x)
+    if codes is None:
+        codes = empty_codes(fmt, rows, cols, x.device)
+    if scales is None:
+        scales = torch.empty(mxq_mma_scales_bytes(rows, cols), dtype=torch.uint8, device=x.device)
+    _check(mxq_quantize_mma(_fmt(fmt), x.data_ptr(), _dt(x), rows, cols, codes.data_ptr(), scales.data_ptr(),
+                            _stream(stream)), "mxq_quantize_mma")
+    return codes, scales
+
+
+def swizzle_scales(scales, out=None, stream=None):
+    """uint8 scales [rows, kblocks] (contiguous, CUDA) -> 1-D uint8 tensor in the MMA tile layout."""
+    torch = _torch()
+    if scales.dtype != torch.uint8 or scales.dim() != 2 or not scales.is_contiguous():
+        raise ValueError("scales must be a contiguous 2-D uint8 tensor")
+    rows, kb = scales.shape
+    if out is None:
+        out = torch.empty(mxq_mma_scales_bytes(rows, 32 * kb), dtype=torch.uint8, device=scales.device)
+    _check(mxq_swizzle_scales(scales.data_ptr(), rows, kb, out.data_ptr(), _stream(stream)), "mxq_swizzle_scales")
+    return out
 
 
 def quantize_grouped(xs, fmt, outs=None, stream=None):

@@ -199,6 +199,41 @@ MXQ_API mxq_status mxq_dequantize_exmy(int ebits, int mbits, const void* codes, 
 MXQ_API mxq_status mxq_fake_quantize_exmy(int ebits, int mbits, const void* src, mxq_dtype dtype, int64_t rows,
                                           int64_t cols, void* dst, mxq_stream stream);
 
+/*
+ * Scale layout of the block-scaled tensor-core MMA. Converted weights are
+ * operands of block-scaled GEMMs ("Sonar: Online MXFP6", Current limits: dense
+ * dimensions in multiples of 128). The pages do not spell out how those GEMMs
+ * read the scales; this is the layout of the sm_100 block-scaled MMA and of
+ * cuBLAS's block-scaled GEMMs ("1D block scaling factors layout"):
+ *   the [rows, kb] E8M0 scale matrix of an operand [rows, K] (kb = K / 32) is
+ *   padded with zero bytes to rows128 = ceil(rows/128)*128 rows and
+ *   kb4 = ceil(kb/4)*4 columns and cut into 128 x 4 tiles of 512 bytes,
+ *   stored tile-row by tile-row (tile (R, C) at byte (R * kb4/4 + C) * 512);
+ *   inside a tile, row r and column c sit at byte (r % 32) * 16 + (r / 32) * 4 + c.
+ * The codes of an MXFP8 E4M3 operand are then exactly a row-major
+ * float8_e4m3fn [rows, K] matrix, those of MXFP4 a row-major packed
+ * float4_e2m1 [rows, K/2] matrix (element 2i in the low nibble).
+ */
+/* Bytes of the tiled scale array of a [rows, cols] operand: rows128 * kb4
+ * (0 on bad input: rows < 0, cols <= 0 or cols % 32 != 0). */
+MXQ_API size_t mxq_mma_scales_bytes(int64_t rows, int64_t cols);
+/* mxq_quantize with the scales written in the tiled layout above. Codes are
+ * identical to mxq_quantize's. scales: device, mxq_mma_scales_bytes(rows, cols)
+ * bytes, written in full: when rows % 128 or (cols/32) % 4 is nonzero the pad
+ * bytes are zeroed by a cudaMemsetAsync on the same stream before the kernel.
+ * E8M0 formats only: MXQ_AXS6 (whose header is 16 bits) -> MXQ_ERR_UNSUPPORTED.
+ * Other rules, errors and overlap checks as mxq_quantize. */
+MXQ_API mxq_status mxq_quantize_mma(mxq_format fmt, const void* src, mxq_dtype dtype, int64_t rows, int64_t cols,
+                                    void* codes, void* scales, mxq_stream stream);
+/* Rearrange a plain scale array (uint8 [rows, kblocks], as written by
+ * mxq_quantize, mxq_exp_quantize or mxq_quantize_cols for its transposed
+ * operand) into the tiled layout. out: device, 4-byte aligned,
+ * mxq_mma_scales_bytes(rows, 32 * kblocks) bytes, all written (pad = 0); it
+ * may not overlap scales. rows == 0 is a no-op; rows < 0 or kblocks <= 0 ->
+ * MXQ_ERR_SHAPE. */
+MXQ_API mxq_status mxq_swizzle_scales(const void* scales, int64_t rows, int64_t kblocks, void* out,
+                                      mxq_stream stream);
+
 /* Bytes of the packed code array: rows * cols/32 * payload (0 on bad input). */
 MXQ_API size_t mxq_codes_bytes(mxq_format fmt, int64_t rows, int64_t cols);
 /* Bytes of the scale array: rows * cols/32 (x2 for AXS-6 headers; 0 on bad input). */

@@ -30,7 +30,7 @@ def declared_symbols():
 
 def test_exports_every_declared_symbol(L):
     syms = declared_symbols()
-    assert len(syms) == 15
+    assert len(syms) == 18
     out = subprocess.run(["nm", "-D", "--defined-only", mxq.LIB_PATH], capture_output=True, text=True).stdout
     exported = set(re.findall(r"\bT\s+(mxq_\w+)", out))
     for s in syms:
@@ -86,10 +86,24 @@ def test_statuses_before_any_cuda_call(L):
     assert mxq.mxq_quantize_grouped(1, 1, [], None) == 1
     assert mxq.mxq_quantize_grouped(1, 1, [(0, 0, 0, 0, 64)], None) == 0
     assert mxq.mxq_quantize_grouped(1, 1, [(0, 0, 0, 0, 64)] * 65, None) == 1
+    assert mxq.mxq_quantize_mma(0, None, 1, 128, 128, None, None, None) == 4   # AXS-6 header is 16 bits
+    assert mxq.mxq_quantize_mma(1, None, 1, 128, 100, None, None, None) == 2
+    assert mxq.mxq_quantize_mma(3, None, 1, 0, 128, None, None, None) == 0
+    assert mxq.mxq_quantize_mma(3, None, 1, 1, 128, None, None, None) == 1
+    assert mxq.mxq_swizzle_scales(None, -1, 4, None, None) == 2
+    assert mxq.mxq_swizzle_scales(None, 4, 0, None, None) == 2
+    assert mxq.mxq_swizzle_scales(None, 0, 4, None, None) == 0
+    assert mxq.mxq_swizzle_scales(None, 4, 4, None, None) == 1
     for s in range(7):
         assert mxq.mxq_status_string(s)
     assert mxq.mxq_status_string(99) == "unknown status"
     assert mxq.mxq_version().count(".") == 2
+
+
+def test_mma_scales_bytes_match_oracle(L):
+    for rows, cols in [(1, 32), (127, 96), (128, 128), (129, 160), (4096, 4096), (0, 64)]:
+        assert mxq.mxq_mma_scales_bytes(rows, cols) == oracle.mma_scales_bytes(rows, cols // 32)
+    assert mxq.mxq_mma_scales_bytes(4, 33) == 0 and mxq.mxq_mma_scales_bytes(-1, 32) == 0
 
 
 def test_block_size_other_than_32_is_rejected():
