@@ -92,6 +92,35 @@ mxq_status check_quantize_args(mxq_format fmt, const void* src, mxq_dtype dtype,
     return MXQ_OK;
 }
 
+mxq_status check_dequantize_args(mxq_format fmt, const void* codes, const void* scales, int64_t rows, int64_t cols,
+                                 void* dst, mxq_dtype dtype) {
+    if (!fmt_ok(fmt) || !dtype_ok(dtype)) return MXQ_ERR_INVALID_ARG;
+    MXQ_TRY(check_shape(rows, cols));
+    if (rows == 0) return MXQ_OK;
+    MXQ_TRY(check_ptr(codes, 16));
+    MXQ_TRY(check_ptr(scales, scales_align(fmt)));
+    MXQ_TRY(check_ptr(dst, 16));
+    const size_t nd = (size_t)rows * (size_t)cols * dtype_bytes(dtype);
+    if (overlap(dst, nd, codes, codes_bytes(fmt, rows, cols)) || overlap(dst, nd, scales, scales_bytes(fmt, rows, cols)))
+        return MXQ_ERR_INVALID_ARG;
+    return MXQ_OK;
+}
+
+mxq_status check_fake_args(mxq_format fmt, const void* src, mxq_dtype dtype, int64_t rows, int64_t cols, void* dst) {
+    if (!fmt_ok(fmt) || !dtype_ok(dtype)) return MXQ_ERR_INVALID_ARG;
+    MXQ_TRY(check_shape(rows, cols));
+    if (rows == 0) return MXQ_OK;
+    MXQ_TRY(check_ptr(src, 16));
+    MXQ_TRY(check_ptr(dst, 16));
+    const size_t nb = (size_t)rows * (size_t)cols * dtype_bytes(dtype);
+    if (src != dst && overlap(src, nb, dst, nb)) return MXQ_ERR_INVALID_ARG;
+    return MXQ_OK;
+}
+
+bool aligned32(const void* a, const void* b) {
+    return ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b)) & 31) == 0;
+}
+
 }  // namespace
 
 extern "C" {
@@ -165,30 +194,87 @@ mxq_status mxq_quantize_grouped(mxq_format fmt, mxq_dtype dtype, const mxq_tenso
 
 mxq_status mxq_dequantize(mxq_format fmt, const void* codes, const void* scales, int64_t rows, int64_t cols,
                           void* dst, mxq_dtype dtype, mxq_stream stream) {
-    if (!fmt_ok(fmt) || !dtype_ok(dtype)) return MXQ_ERR_INVALID_ARG;
-    MXQ_TRY(check_shape(rows, cols));
+    MXQ_TRY(check_dequantize_args(fmt, codes, scales, rows, cols, dst, dtype));
     if (rows == 0) return MXQ_OK;
-    MXQ_TRY(check_ptr(codes, 16));
-    MXQ_TRY(check_ptr(scales, scales_align(fmt)));
-    MXQ_TRY(check_ptr(dst, 16));
-    const size_t nd = (size_t)rows * (size_t)cols * dtype_bytes(dtype);
-    if (overlap(dst, nd, codes, codes_bytes(fmt, rows, cols)) || overlap(dst, nd, scales, scales_bytes(fmt, rows, cols)))
-        return MXQ_ERR_INVALID_ARG;
     return from_cuda(mxq::launch_dequantize((int)fmt, codes, scales, dst, (int)dtype, rows * (cols / 32),
                                             (cudaStream_t)stream));
 }
 
 mxq_status mxq_fake_quantize(mxq_format fmt, const void* src, mxq_dtype dtype, int64_t rows, int64_t cols, void* dst,
                              mxq_stream stream) {
-    if (!fmt_ok(fmt) || !dtype_ok(dtype)) return MXQ_ERR_INVALID_ARG;
-    MXQ_TRY(check_shape(rows, cols));
+    MXQ_TRY(check_fake_args(fmt, src, dtype, rows, cols, dst));
     if (rows == 0) return MXQ_OK;
-    MXQ_TRY(check_ptr(src, 16));
-    MXQ_TRY(check_ptr(dst, 16));
-    const size_t nb = (size_t)rows * (size_t)cols * dtype_bytes(dtype);
-    if (src != dst && overlap(src, nb, dst, nb)) return MXQ_ERR_INVALID_ARG;
     return from_cuda(mxq::launch_fake_quantize((int)fmt, src, dst, (int)dtype, rows * (cols / 32),
                                                (cudaStream_t)stream));
+}
+
+mxq_status mxq_run_batch(mxq_dtype dtype, const mxq_op* ops, int n, mxq_stream stream) {
+    if (!dtype_ok(dtype) || ops == nullptr || n < 1 || n > MXQ_MAX_BATCH) return MXQ_ERR_INVALID_ARG;
+    struct Range {
+        const void* p;
+        size_t n;
+    };
+    Range rin[MXQ_MAX_BATCH][2], rout[MXQ_MAX_BATCH][2];
+    mxq::BatchTable tab{};
+    int m = 0;
+    for (int i = 0; i < n; ++i) {
+        const mxq_op& o = ops[i];
+        const mxq_format f = (mxq_format)o.fmt;
+        if (!fmt_ok(f)) return MXQ_ERR_INVALID_ARG;
+        const size_t nv = (size_t)o.rows * (size_t)(o.cols > 0 ? o.cols : 0) * dtype_bytes(dtype);
+        mxq::BatchOp b{};
+        b.kind = o.kind;
+        b.fmt = o.fmt;
+        b.nblocks = o.rows * (o.cols / 32);
+        if (o.kind == MXQ_OP_QUANTIZE) {
+            MXQ_TRY(check_quantize_args(f, o.src, dtype, o.rows, o.cols, o.dst, o.dst_scales));
+            b.in = o.src;
+            b.out = o.dst;
+            b.scales_out = o.dst_scales;
+            rin[m][0] = {o.src, nv};
+            rin[m][1] = {nullptr, 0};
+            rout[m][0] = {o.dst, codes_bytes(f, o.rows, o.cols)};
+            rout[m][1] = {o.dst_scales, scales_bytes(f, o.rows, o.cols)};
+        } else if (o.kind == MXQ_OP_DEQUANTIZE) {
+            MXQ_TRY(check_dequantize_args(f, o.src, o.src_scales, o.rows, o.cols, o.dst, dtype));
+            b.in = o.src;
+            b.scales_in = o.src_scales;
+            b.out = o.dst;
+            rin[m][0] = {o.src, codes_bytes(f, o.rows, o.cols)};
+            rin[m][1] = {o.src_scales, scales_bytes(f, o.rows, o.cols)};
+            rout[m][0] = {o.dst, nv};
+            rout[m][1] = {nullptr, 0};
+        } else if (o.kind == MXQ_OP_FAKE_QUANTIZE) {
+            MXQ_TRY(check_fake_args(f, o.src, dtype, o.rows, o.cols, o.dst));
+            b.in = o.src;
+            b.out = o.dst;
+            rin[m][0] = {o.src, nv};
+            rin[m][1] = {nullptr, 0};
+            rout[m][0] = {o.dst, nv};
+            rout[m][1] = {nullptr, 0};
+        } else {
+            return MXQ_ERR_INVALID_ARG;
+        }
+        if (o.rows == 0) continue;
+        b.a32 = aligned32(b.in, b.out) ? 1 : 0;
+        tab.op[m++] = b;
+    }
+    // the ops run concurrently: an op's outputs may not touch another op's inputs or outputs
+    for (int i = 0; i < m; ++i)
+        for (int j = 0; j < m; ++j) {
+            if (i == j) continue;
+            for (int a = 0; a < 2; ++a)
+                for (int c = 0; c < 2; ++c) {
+                    const Range& w = rout[i][a];
+                    if (w.n == 0) continue;
+                    if ((rin[j][c].n && overlap(w.p, w.n, rin[j][c].p, rin[j][c].n)) ||
+                        (rout[j][c].n && overlap(w.p, w.n, rout[j][c].p, rout[j][c].n)))
+                        return MXQ_ERR_INVALID_ARG;
+                }
+        }
+    if (m == 0) return MXQ_OK;
+    tab.n = m;
+    return from_cuda(mxq::launch_batch((int)dtype, tab, (cudaStream_t)stream));
 }
 
 mxq_status mxq_exp_quantize(mxq_format fmt, const float* scores, int64_t rows, int64_t cols, void* codes,

@@ -56,25 +56,6 @@ template <int F, typename T, int NSEG> __host__ __device__ constexpr bool q_stag
     return NSEG == 1 && Fmt<F>::W == 6 && !Fmt<F>::FIXED;
 }
 
-// 6-bit payloads are 24 bytes: a warp's 32 consecutive blocks are assembled in
-// shared memory and leave as 16-byte stores (48 of them) instead of 3 x 8 bytes
-// per thread.
-template <int F>
-__device__ __forceinline__ void warp_store6(void* codes, long long first_blk, int nvalid, const uint32_t* out,
-                                            uint8_t* stage, int lane) {
-    uint2* q = reinterpret_cast<uint2*>(stage + 24 * lane);
-    q[0] = make_uint2(out[0], out[1]);
-    q[1] = make_uint2(out[2], out[3]);
-    q[2] = make_uint2(out[4], out[5]);
-    __syncwarp();
-    char* g = reinterpret_cast<char*>(codes) + first_blk * 24;
-    const int nbytes = 24 * nvalid;
-    for (int i = 16 * lane; i + 16 <= nbytes; i += 512)
-        st_stream_v4(g + i, *reinterpret_cast<const uint4*>(stage + i));
-    if ((nbytes & 15) && lane == 0) *reinterpret_cast<uint2*>(g + (nbytes & ~15)) = *reinterpret_cast<const uint2*>(stage + (nbytes & ~15));
-    __syncwarp();
-}
-
 // MMA: scales go to the block-scaled MMA tile layout (single tensor, E8M0 formats); a separate
 // instantiation, so the plain and grouped kernels carry no trace of it.
 template <int F, typename T, int NSEG, bool MMA = false>
@@ -184,7 +165,7 @@ __global__ void __launch_bounds__(kThreads) k_fake_quantize(const void* src, voi
 // launchers
 
 // Resident CTAs per SM (occupancy query) times the SM count, cached per kernel and device.
-static int resident_ctas(const void* fn, int dev) {
+int resident_ctas(const void* fn, int dev) {
     struct Entry { const void* fn; int dev; int ctas; };
     static Entry cache[512];
     static int used = 0;

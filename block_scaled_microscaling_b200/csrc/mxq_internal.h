@@ -8,6 +8,9 @@ namespace mxq {
 
 constexpr int kMaxSeg = 64;  // == MXQ_MAX_GROUP
 
+// SMs x resident CTAs of 256 threads for a kernel (occupancy query, cached per kernel and device)
+int resident_ctas(const void* fn, int dev);
+
 // one tensor of a (grouped) quantize launch
 struct Seg {
     const void* src;
@@ -22,6 +25,26 @@ template <int N> struct SegTable {
     int n;
     long long nblocks;  // all tensors' blocks
 };
+
+// one conversion of a batch launch: kind 0 quantize (in values -> out codes, scales_out),
+// 1 dequantize (in codes + scales_in -> out values), 2 fake-quantize (in values -> out values)
+struct BatchOp {
+    int kind;
+    int fmt;
+    int a32;            // in and out both 32-byte aligned: 256-bit accesses
+    const void* in;
+    const void* scales_in;
+    void* out;
+    void* scales_out;
+    long long nblocks;  // blocks of 32 values
+    long long tile0;    // first warp tile (32 blocks) of this op in the batch (filled by the launcher)
+};
+struct BatchTable {
+    BatchOp op[kMaxSeg];
+    int n;
+    long long ntiles;
+};
+cudaError_t launch_batch(int dtype, BatchTable& tab, cudaStream_t st);
 
 // fmt: 0 AXS-6, 1 E2M3, 2 E3M2, 3 E4M3, 4 E2M1; dtype: 0 fp32, 1 bf16
 template <int NSEG>

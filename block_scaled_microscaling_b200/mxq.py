@@ -24,7 +24,7 @@ ELEM_BITS = {"axs6": 6, "mxfp6_e2m3": 6, "mxfp6_e3m2": 6, "mxfp8": 8, "mxfp4": 4
 
 EXPORTS = ["mxq_quantize", "mxq_dequantize", "mxq_fake_quantize", "mxq_exp_quantize", "mxq_quantize_grouped",
            "mxq_quantize_cols", "mxq_dequantize_cols", "mxq_quantize_exmy", "mxq_dequantize_exmy",
-           "mxq_fake_quantize_exmy", "mxq_quantize_mma", "mxq_swizzle_scales", "mxq_mma_scales_bytes",
+           "mxq_fake_quantize_exmy", "mxq_quantize_mma", "mxq_swizzle_scales", "mxq_mma_scales_bytes", "mxq_run_batch",
            "mxq_codes_bytes", "mxq_scales_bytes", "mxq_block_bits", "mxq_status_string",
            "mxq_version"]
 
@@ -37,6 +37,12 @@ class MXQError(RuntimeError):
 
 class _Tensor(ctypes.Structure):
     _fields_ = [("src", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
+
+
+class _Op(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("fmt", ctypes.c_int), ("src", ctypes.c_void_p),
+                ("src_scales", ctypes.c_void_p), ("dst", ctypes.c_void_p), ("dst_scales", ctypes.c_void_p),
                 ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
 
 
@@ -64,6 +70,7 @@ def lib():
             ("mxq_dequantize_exmy", [i32, i32, vp, vp, i64, i64, vp, i32, vp]),
             ("mxq_fake_quantize_exmy", [i32, i32, vp, i32, i64, i64, vp, vp]),
             ("mxq_quantize_mma", [i32, vp, i32, i64, i64, vp, vp, vp]),
+            ("mxq_run_batch", [i32, ctypes.POINTER(_Op), i32, vp]),
             ("mxq_swizzle_scales", [vp, i64, i64, vp, vp]),
         ]:
             fn = getattr(L, name)
@@ -141,6 +148,14 @@ def mxq_swizzle_scales(scales, rows, kblocks, out, stream):
 
 def mxq_mma_scales_bytes(rows, cols):
     return lib().mxq_mma_scales_bytes(rows, cols)
+
+
+def mxq_run_batch(dtype, ops, stream):
+    """ops: sequence of (kind, fmt, src, src_scales, dst, dst_scales, rows, cols) integer tuples."""
+    arr = (_Op * max(1, len(ops)))()
+    for i, o in enumerate(ops):
+        arr[i] = _Op(*o)
+    return lib().mxq_run_batch(dtype, arr, len(ops), stream)
 
 
 def mxq_codes_bytes(fmt, rows, cols):
@@ -300,6 +315,42 @@ def swizzle_scales(scales, out=None, stream=None):
         out = torch.empty(mxq_mma_scales_bytes(rows, 32 * kb), dtype=torch.uint8, device=scales.device)
     _check(mxq_swizzle_scales(scales.data_ptr(), rows, kb, out.data_ptr(), _stream(stream)), "mxq_swizzle_scales")
     return out
+
+
+OP_KINDS = {"quantize": 0, "dequantize": 1, "fake_quantize": 2}
+
+
+def batch(ops, stream=None):
+    """Several independent conversions in one launch (all values of one dtype):
+      ("quantize", fmt, x, codes, scales)
+      ("dequantize", fmt, codes, scales, out)      -- out's shape gives rows, cols
+      ("fake_quantize", fmt, x, out)
+    Outputs must be preallocated; no output may overlap another op's buffers."""
+    descs, dtype = [], None
+    for op in ops:
+        kind = op[0]
+        if kind == "quantize":
+            _, fmt, x, codes, scales = op
+            vals, d = x, (x.data_ptr(), 0, codes.data_ptr(), scales.data_ptr())
+        elif kind == "dequantize":
+            _, fmt, codes, scales, out = op
+            vals, d = out, (codes.data_ptr(), scales.data_ptr(), out.data_ptr(), 0)
+        elif kind == "fake_quantize":
+            _, fmt, x, out = op
+            vals, d = x, (x.data_ptr(), 0, out.data_ptr(), 0)
+        else:
+            raise ValueError(f"unknown batch op {kind!r}")
+        if not vals.is_contiguous():
+            raise ValueError("value tensors must be contiguous")
+        if dtype is None:
+            dtype = _dt(vals)
+        elif _dt(vals) != dtype:
+            raise TypeError("all values of a batch must have one dtype")
+        rows, cols = _as2d(vals)
+        descs.append((OP_KINDS[kind], _fmt(fmt), *d, rows, cols))
+    if not descs:
+        raise ValueError("empty batch")
+    _check(mxq_run_batch(dtype, descs, _stream(stream)), "mxq_run_batch")
 
 
 def quantize_grouped(xs, fmt, outs=None, stream=None):

@@ -200,6 +200,37 @@ MXQ_API mxq_status mxq_fake_quantize_exmy(int ebits, int mbits, const void* src,
                                           int64_t cols, void* dst, mxq_stream stream);
 
 /*
+ * Batch: n independent conversions on one value type in a single launch, for
+ * example the tensors of one layer going to the formats a per-module policy
+ * chose ("Sonar: Online MXFP6", Start a model and Select the FP6 encoding), or
+ * weights dequantized beside activations quantized. Results are bit-identical
+ * to the single-operation entry points; the batch pays one launch instead of n.
+ *   kind MXQ_OP_QUANTIZE:      src = values [rows, cols] (dtype), dst = codes,
+ *                              dst_scales = scales (mxq_quantize's layouts)
+ *   kind MXQ_OP_DEQUANTIZE:    src = codes, src_scales = scales, dst = values
+ *   kind MXQ_OP_FAKE_QUANTIZE: src = values, dst = values (dst == src allowed)
+ * Unused pointer fields are ignored. Each op obeys the shape, alignment and
+ * overlap rules of its single-operation entry point. The ops run concurrently,
+ * so no op may write memory that another op of the batch reads or writes
+ * (MXQ_ERR_INVALID_ARG otherwise). 1 <= n <= MXQ_MAX_BATCH; ops with rows == 0
+ * are skipped. The descriptor array is read on the host during the call only.
+ */
+typedef enum { MXQ_OP_QUANTIZE = 0, MXQ_OP_DEQUANTIZE = 1, MXQ_OP_FAKE_QUANTIZE = 2 } mxq_op_kind;
+#define MXQ_MAX_BATCH 64
+typedef struct {
+    int kind;               /* mxq_op_kind */
+    int fmt;                /* mxq_format */
+    const void* src;
+    const void* src_scales;
+    void* dst;
+    void* dst_scales;
+    int64_t rows;
+    int64_t cols;
+} mxq_op;
+
+MXQ_API mxq_status mxq_run_batch(mxq_dtype dtype, const mxq_op* ops, int n, mxq_stream stream);
+
+/*
  * Scale layout of the block-scaled tensor-core MMA. Converted weights are
  * operands of block-scaled GEMMs ("Sonar: Online MXFP6", Current limits: dense
  * dimensions in multiples of 128). The pages do not spell out how those GEMMs

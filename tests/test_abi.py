@@ -30,7 +30,7 @@ def declared_symbols():
 
 def test_exports_every_declared_symbol(L):
     syms = declared_symbols()
-    assert len(syms) == 18
+    assert len(syms) == 19
     out = subprocess.run(["nm", "-D", "--defined-only", mxq.LIB_PATH], capture_output=True, text=True).stdout
     exported = set(re.findall(r"\bT\s+(mxq_\w+)", out))
     for s in syms:
@@ -44,10 +44,13 @@ def test_enum_values_match_header():
     for name, v in [("MXQ_AXS6", 0), ("MXQ_MXFP6_E2M3", 1), ("MXQ_MXFP6_E3M2", 2), ("MXQ_MXFP8_E4M3", 3),
                     ("MXQ_MXFP4_E2M1", 4), ("MXQ_F32", 0), ("MXQ_BF16", 1), ("MXQ_OK", 0),
                     ("MXQ_ERR_INVALID_ARG", 1), ("MXQ_ERR_SHAPE", 2), ("MXQ_ERR_ALIGN", 3),
-                    ("MXQ_ERR_UNSUPPORTED", 4), ("MXQ_ERR_CUDA", 5), ("MXQ_ERR_TIMEOUT", 6)]:
+                    ("MXQ_ERR_UNSUPPORTED", 4), ("MXQ_ERR_CUDA", 5), ("MXQ_ERR_TIMEOUT", 6),
+                    ("MXQ_OP_QUANTIZE", 0), ("MXQ_OP_DEQUANTIZE", 1), ("MXQ_OP_FAKE_QUANTIZE", 2)]:
         assert re.search(rf"\b{name}\s*=\s*{v}\b", src), name
     assert list(mxq.FORMATS.values()) == [0, 1, 2, 3, 4]
     assert re.search(r"#define MXQ_MAX_GROUP\s+(\d+)", src).group(1) == str(mxq.MAX_GROUP)
+    assert re.search(r"#define MXQ_MAX_BATCH\s+(\d+)", src).group(1) == "64"
+    assert mxq.OP_KINDS == {"quantize": 0, "dequantize": 1, "fake_quantize": 2}
 
 
 def test_block_bits_match_page_facts(L):
@@ -94,6 +97,15 @@ def test_statuses_before_any_cuda_call(L):
     assert mxq.mxq_swizzle_scales(None, 4, 0, None, None) == 2
     assert mxq.mxq_swizzle_scales(None, 0, 4, None, None) == 0
     assert mxq.mxq_swizzle_scales(None, 4, 4, None, None) == 1
+    b = mxq.mxq_run_batch
+    assert b(1, [], None) == 1                                          # n = 0
+    assert b(1, [(0, 1, 0, 0, 0, 0, 0, 64)] * 65, None) == 1            # n > 64
+    assert b(1, [(3, 1, 0, 0, 0, 0, 0, 64)], None) == 1                 # bad kind
+    assert b(1, [(0, 9, 0, 0, 0, 0, 0, 64)], None) == 1                 # bad format
+    assert b(7, [(0, 1, 0, 0, 0, 0, 0, 64)], None) == 1                 # bad dtype
+    assert b(1, [(1, 1, 0, 0, 0, 0, 2, 48)], None) == 2                 # cols % 32
+    assert b(1, [(0, 1, 0, 0, 0, 0, 0, 64), (2, 0, 0, 0, 0, 0, 0, 32)], None) == 0  # all empty
+    assert b(1, [(0, 1, 0, 0, 0, 0, 1, 64)], None) == 1                 # null pointers
     for s in range(7):
         assert mxq.mxq_status_string(s)
     assert mxq.mxq_status_string(99) == "unknown status"
