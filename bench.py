@@ -54,27 +54,34 @@ def peaks():
     return FALLBACK_HBM, "fallback"
 
 
-def ncu_traffic(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu capture, or None when
-    the kernel sources have changed since that capture (or it was not captured)."""
-    import glob
+def sources_sha256(names):
+    """sha256 over the named files of the kernel sources (name + contents, in the given order)."""
     import hashlib
+    csrc = os.path.join(ROOT, "block_scaled_microscaling_b200", "csrc")
+    h = hashlib.sha256()
+    for nm in names:
+        h.update(nm.encode())
+        with open(os.path.join(csrc, nm), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture, or None when the
+    kernel's source files have changed since that capture (or it was not captured)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
-        d = json.load(f)
-    csrc = os.path.join(ROOT, "block_scaled_microscaling_b200", "csrc")
-    h = hashlib.sha256()
-    for fn in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")) +
-                     glob.glob(os.path.join(csrc, "*.h"))):
-        h.update(os.path.basename(fn).encode())
-        with open(fn, "rb") as f:
-            h.update(f.read())
-    if h.hexdigest() != d.get("csrc_sha256"):
+        e = json.load(f).get("kernels", {}).get(kernel)
+    if not e:
         return None
-    v = d.get("bytes_per_launch", {}).get(kernel)
-    return int(v) if v is not None else None
+    try:
+        if sources_sha256(e["sources"]) != e["sources_sha256"]:
+            return None
+    except OSError:
+        return None
+    return int(e["bytes_per_launch"])
 
 
 def nbytes_q(fmt, n_elems, in_bytes):

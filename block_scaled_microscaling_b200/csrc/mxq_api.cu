@@ -277,6 +277,21 @@ mxq_status mxq_run_batch(mxq_dtype dtype, const mxq_op* ops, int n, mxq_stream s
     return from_cuda(mxq::launch_batch((int)dtype, tab, (cudaStream_t)stream));
 }
 
+mxq_status mxq_check_device(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return MXQ_ERR_CUDA;
+    unsigned int v = 0;
+    if (mxq::read_device_error(&v, true) != cudaSuccess) return MXQ_ERR_CUDA;
+    return v ? MXQ_ERR_TIMEOUT : MXQ_OK;
+}
+
+mxq_status mxq_selftest_timeout(int limit_ms) {
+    if (limit_ms < 1 || limit_ms > 1000) return MXQ_ERR_INVALID_ARG;
+    const mxq_status before = mxq_check_device();  // start from a clear word
+    if (before == MXQ_ERR_CUDA) return before;
+    if (mxq::launch_selftest_timeout((unsigned long long)limit_ms * 1000000ull, 0) != cudaSuccess) return MXQ_ERR_CUDA;
+    return mxq_check_device();
+}
+
 mxq_status mxq_exp_quantize(mxq_format fmt, const float* scores, int64_t rows, int64_t cols, void* codes,
                             void* scales, mxq_stream stream) {
     MXQ_TRY(check_quantize_args(fmt, scores, MXQ_F32, rows, cols, codes, scales));

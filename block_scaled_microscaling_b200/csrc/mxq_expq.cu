@@ -12,104 +12,17 @@
 // L2, the second re-reads it from L2 and exponentiates and quantizes each
 // 32-key block in registers. The launcher keeps the rows in flight within half
 // of L2, so HBM sees each score once. Any row length (cols % 32 == 0).
+// MXFP4 and MXFP8 take the bulk-copy pipeline of mxq_expq_tma.cu instead; this
+// kernel serves the 6-bit formats.
 #include <cstdint>
 #include <cuda_runtime.h>
 
 #include "mxq_block.cuh"
 #include "mxq_device.cuh"
+#include "mxq_exp.cuh"
 #include "mxq_internal.h"
 
 namespace mxq {
-
-
-// The library's own fp32 exponential (the same definition the CPU oracle
-// implements independently):
-//   t = RN(d * L2E), n = t rounded to an integer, ties to even,
-//   r = RN(d - n*LN2_HI) and r = RN(r - n*LN2_LO), both fused (Cody & Waite),
-//   p = Horner over 1/k!, k = 7..0, one fused multiply-add per step,
-//   e^d = p * 2^n (outside 2^[-126,127] as two exact-then-rounded products
-//   through 2^(n+-64)); t < -160 -> +0, t > 160 -> +inf, NaN -> NaN.
-// L2E = 1/ln2 and LN2_LO = ln2 - LN2_HI rounded to fp32, LN2_HI = ln 2 cut to
-// 16 significant bits, 1/k! rounded to fp32.
-constexpr float kL2E = 0x1.715476p+0f, kLn2Hi = 0x1.62e4p-1f, kLn2Lo = 0x1.7f7d1cp-20f;
-constexpr float kC0 = 0x1p+0f, kC1 = 0x1p+0f, kC2 = 0x1p-1f, kC3 = 0x1.555556p-3f, kC4 = 0x1.555556p-5f,
-                kC5 = 0x1.111112p-7f, kC6 = 0x1.6c16c2p-10f, kC7 = 0x1.a01a02p-13f;
-constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer (|x| < 2^22)
-
-__device__ __forceinline__ float pow2i(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
-
-// general form, any input
-__device__ __forceinline__ float expf_mxq(float d) {
-    if (d != d) return d;
-    float t = __fmul_rn(d, kL2E);
-    if (t < -160.0f) return 0.0f;
-    if (t > 160.0f) return __uint_as_float(0x7F800000u);
-    float n = __fsub_rn(__fadd_rn(t, kRound), kRound);  // rint(t), ties to even
-    float r = __fmaf_rn(-n, kLn2Hi, d);
-    r = __fmaf_rn(-n, kLn2Lo, r);
-    float p = kC7;
-    p = __fmaf_rn(p, r, kC6);
-    p = __fmaf_rn(p, r, kC5);
-    p = __fmaf_rn(p, r, kC4);
-    p = __fmaf_rn(p, r, kC3);
-    p = __fmaf_rn(p, r, kC2);
-    p = __fmaf_rn(p, r, kC1);
-    p = __fmaf_rn(p, r, kC0);
-    int ni = (int)n;
-    if (ni < -126) return __fmul_rn(__fmul_rn(p, pow2i(ni + 64)), pow2i(-64));
-    if (ni > 127) return __fmul_rn(__fmul_rn(p, pow2i(ni - 64)), pow2i(64));
-    return __fmul_rn(p, pow2i(ni));
-}
-
-// Same function on a packed pair of shifted scores d = (lo, hi), valid when both
-// t = d*L2E lie in [-126, 127] (then 2^n is one normal fp32 and one product
-// suffices): n from the 1.5*2^23 add, 2^n's bits from that sum's bits.
-__device__ __forceinline__ unsigned long long expf_mxq2(unsigned long long d) {
-    const unsigned long long tm = f2add(f2mul(d, dup2(kL2E)), dup2(kRound));
-    const unsigned long long nn = f2sub(dup2(kRound), tm);  // -n, exact
-    unsigned long long r = f2fma(nn, dup2(kLn2Hi), d);
-    r = f2fma(nn, dup2(kLn2Lo), r);
-    unsigned long long p = f2fma(dup2(kC7), r, dup2(kC6));
-    p = f2fma(p, r, dup2(kC5));
-    p = f2fma(p, r, dup2(kC4));
-    p = f2fma(p, r, dup2(kC3));
-    p = f2fma(p, r, dup2(kC2));
-    p = f2fma(p, r, dup2(kC1));
-    p = f2fma(p, r, dup2(kC0));
-    float a, b;
-    upk(tm, a, b);
-    // bits(tm) = 0x4B400000 + n, so (n + 127) << 23 = bits(tm) * 2^23 + 0x3F800000 (mod 2^32)
-    const float sa = __uint_as_float(__float_as_uint(a) * 0x800000u + 0x3F800000u);
-    const float sb = __uint_as_float(__float_as_uint(b) * 0x800000u + 0x3F800000u);
-    return f2mul(p, pk(sa, sb));
-}
-
-// Shifted scores d = x - mr -> e^d, in place, for n values (n even); packed
-// path unless some t = d*L2E < -126 among them.
-template <int N>
-__device__ __forceinline__ void exp_values(uint32_t (&w)[N], float mr) {
-    float tmin = 0.0f;
-#pragma unroll
-    for (int i = 0; i < N / 2; ++i) {
-        float a, b;
-        upk(f2sub(pk(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1])), dup2(mr)), a, b);
-        w[2 * i] = __float_as_uint(a);
-        w[2 * i + 1] = __float_as_uint(b);
-        tmin = min3f(tmin, a, b);
-    }
-    if (__fmul_rn(tmin, kL2E) >= -126.0f) {
-#pragma unroll
-        for (int i = 0; i < N / 2; ++i) {
-            float a, b;
-            upk(expf_mxq2(pk(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1]))), a, b);
-            w[2 * i] = __float_as_uint(a);
-            w[2 * i + 1] = __float_as_uint(b);
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < N; ++i) w[i] = __float_as_uint(expf_mxq(__uint_as_float(w[i])));
-    }
-}
 
 
 template <int F>
@@ -244,6 +157,8 @@ static cudaError_t launch_xq(const float* scores, long long rows, long long cols
 cudaError_t launch_exp_quantize(int fmt, const float* scores, long long rows, long long cols, void* codes,
                                 void* scales, cudaStream_t st) {
     if (!exp_quantize_supported(cols)) return cudaErrorNotSupported;
+    if (exp_quantize_tma_supported(fmt, scores))
+        return launch_exp_quantize_tma(fmt, scores, rows, cols, codes, scales, st);
     switch (fmt) {
         case F_AXS6: return launch_xq<F_AXS6>(scores, rows, cols, codes, scales, st);
         case F_E2M3: return launch_xq<F_E2M3>(scores, rows, cols, codes, scales, st);

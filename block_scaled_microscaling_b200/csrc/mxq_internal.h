@@ -57,6 +57,14 @@ cudaError_t launch_fake_quantize(int fmt, const void* src, void* dst, int dtype,
 cudaError_t launch_exp_quantize(int fmt, const float* scores, long long rows, long long cols, void* codes,
                                 void* scales, cudaStream_t st);
 bool exp_quantize_supported(long long cols);
+// bulk-copy pipeline form of the softmax stage (E2M1 and E4M3, scores 16-byte aligned)
+bool exp_quantize_tma_supported(int fmt, const void* scores);
+cudaError_t launch_exp_quantize_tma(int fmt, const float* scores, long long rows, long long cols, void* codes,
+                                    void* scales, cudaStream_t st);
+// the device error word (bit 0: a bounded wait in a kernel ran out); clear resets it
+cudaError_t read_device_error(unsigned int* value, bool clear);
+// one warp waits (bounded by limit_ns) on an mbarrier nothing arrives at
+cudaError_t launch_selftest_timeout(unsigned long long limit_ns, cudaStream_t st);
 // column-direction blocks (32 rows of a column), transposed output layout
 cudaError_t launch_quantize_cols(int fmt, const void* src, int dtype, long long rows, long long cols, void* codes,
                                  void* scales, cudaStream_t st);

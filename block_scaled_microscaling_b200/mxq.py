@@ -24,7 +24,7 @@ ELEM_BITS = {"axs6": 6, "mxfp6_e2m3": 6, "mxfp6_e3m2": 6, "mxfp8": 8, "mxfp4": 4
 
 EXPORTS = ["mxq_quantize", "mxq_dequantize", "mxq_fake_quantize", "mxq_exp_quantize", "mxq_quantize_grouped",
            "mxq_quantize_cols", "mxq_dequantize_cols", "mxq_quantize_exmy", "mxq_dequantize_exmy",
-           "mxq_fake_quantize_exmy", "mxq_quantize_mma", "mxq_swizzle_scales", "mxq_mma_scales_bytes", "mxq_run_batch",
+           "mxq_fake_quantize_exmy", "mxq_quantize_mma", "mxq_swizzle_scales", "mxq_mma_scales_bytes", "mxq_run_batch", "mxq_check_device", "mxq_selftest_timeout",
            "mxq_codes_bytes", "mxq_scales_bytes", "mxq_block_bits", "mxq_status_string",
            "mxq_version"]
 
@@ -80,6 +80,10 @@ def lib():
         L.mxq_codes_bytes.restype = sz
         L.mxq_scales_bytes.argtypes = [i32, i64, i64]
         L.mxq_scales_bytes.restype = sz
+        L.mxq_selftest_timeout.argtypes = [i32]
+        L.mxq_selftest_timeout.restype = i32
+        L.mxq_check_device.argtypes = []
+        L.mxq_check_device.restype = i32
         L.mxq_mma_scales_bytes.argtypes = [i64, i64]
         L.mxq_mma_scales_bytes.restype = sz
         L.mxq_block_bits.argtypes = [i32]
@@ -156,6 +160,19 @@ def mxq_run_batch(dtype, ops, stream):
     for i, o in enumerate(ops):
         arr[i] = _Op(*o)
     return lib().mxq_run_batch(dtype, arr, len(ops), stream)
+
+
+def mxq_check_device():
+    return lib().mxq_check_device()
+
+
+def mxq_selftest_timeout(limit_ms):
+    return lib().mxq_selftest_timeout(limit_ms)
+
+
+def check_device():
+    """Synchronize and raise MXQError(MXQ_ERR_TIMEOUT) if a bounded wait in a kernel ran out."""
+    _check(mxq_check_device(), "mxq_check_device")
 
 
 def mxq_codes_bytes(fmt, rows, cols):

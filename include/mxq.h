@@ -136,6 +136,8 @@ MXQ_API mxq_status mxq_fake_quantize(mxq_format fmt, const void* src, mxq_dtype 
  *   then p is block-quantized exactly like mxq_quantize with dtype MXQ_F32.
  * p is never written to memory. Supported formats: all five (MXFP4 E2M1 is
  * the one the stage feeds). scores 16-byte aligned; any cols % 32 == 0.
+ * MXFP4 and MXFP8 run as a bulk-copy (TMA) pipeline whose waits are bounded;
+ * see mxq_check_device.
  */
 MXQ_API mxq_status mxq_exp_quantize(mxq_format fmt, const float* scores, int64_t rows, int64_t cols,
                             void* codes, void* scales, mxq_stream stream);
@@ -264,6 +266,24 @@ MXQ_API mxq_status mxq_quantize_mma(mxq_format fmt, const void* src, mxq_dtype d
  * MXQ_ERR_SHAPE. */
 MXQ_API mxq_status mxq_swizzle_scales(const void* scales, int64_t rows, int64_t kblocks, void* out,
                                       mxq_stream stream);
+
+/*
+ * Device-side status. The bulk-copy pipeline behind mxq_exp_quantize (MXFP4 /
+ * MXFP8) waits on its own asynchronous copies; every such wait is bounded (one
+ * second). A wait that runs out makes the kernel stop early, leaving its
+ * outputs incomplete, and sets a device error word. mxq_check_device
+ * synchronizes the current device and returns MXQ_ERR_TIMEOUT if that
+ * happened since the last call (clearing the word), MXQ_ERR_CUDA if the device
+ * reported an error, MXQ_OK otherwise. It is host-blocking; call it where a
+ * synchronization is acceptable (after a step, in tests).
+ */
+MXQ_API mxq_status mxq_check_device(void);
+/* Self-test of that mechanism: launches one warp that waits on an mbarrier
+ * nothing arrives at, with a limit of limit_ms milliseconds (1..1000), then
+ * returns mxq_check_device(): MXQ_ERR_TIMEOUT when the wait gave up and was
+ * reported as it should. Synchronizes the device. MXQ_ERR_INVALID_ARG for a
+ * limit out of range. No counterpart on the pages: a diagnostic of the library. */
+MXQ_API mxq_status mxq_selftest_timeout(int limit_ms);
 
 /* Bytes of the packed code array: rows * cols/32 * payload (0 on bad input). */
 MXQ_API size_t mxq_codes_bytes(mxq_format fmt, int64_t rows, int64_t cols);

@@ -30,7 +30,7 @@ def declared_symbols():
 
 def test_exports_every_declared_symbol(L):
     syms = declared_symbols()
-    assert len(syms) == 19
+    assert len(syms) == 21
     out = subprocess.run(["nm", "-D", "--defined-only", mxq.LIB_PATH], capture_output=True, text=True).stdout
     exported = set(re.findall(r"\bT\s+(mxq_\w+)", out))
     for s in syms:
@@ -106,6 +106,7 @@ def test_statuses_before_any_cuda_call(L):
     assert b(1, [(1, 1, 0, 0, 0, 0, 2, 48)], None) == 2                 # cols % 32
     assert b(1, [(0, 1, 0, 0, 0, 0, 0, 64), (2, 0, 0, 0, 0, 0, 0, 32)], None) == 0  # all empty
     assert b(1, [(0, 1, 0, 0, 0, 0, 1, 64)], None) == 1                 # null pointers
+    assert mxq.mxq_selftest_timeout(0) == 1 and mxq.mxq_selftest_timeout(1001) == 1
     for s in range(7):
         assert mxq.mxq_status_string(s)
     assert mxq.mxq_status_string(99) == "unknown status"
