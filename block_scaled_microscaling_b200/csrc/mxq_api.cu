@@ -204,8 +204,8 @@ mxq_status mxq_fake_quantize(mxq_format fmt, const void* src, mxq_dtype dtype, i
                              mxq_stream stream) {
     MXQ_TRY(check_fake_args(fmt, src, dtype, rows, cols, dst));
     if (rows == 0) return MXQ_OK;
-    return from_cuda(mxq::launch_fake_quantize((int)fmt, src, dst, (int)dtype, rows * (cols / 32),
-                                               (cudaStream_t)stream));
+    return from_cuda(mxq::launch_fake_quantize_stream((int)fmt, src, dst, (int)dtype, rows * (cols / 32),
+                                                      (cudaStream_t)stream));
 }
 
 mxq_status mxq_run_batch(mxq_dtype dtype, const mxq_op* ops, int n, mxq_stream stream) {

@@ -37,82 +37,11 @@
 #include "mxq_device.cuh"
 #include "mxq_exp.cuh"
 #include "mxq_internal.h"
+#include "mxq_tma.cuh"
 
 namespace mxq {
 
 __device__ unsigned int g_device_error;  // bit 0: a bounded wait ran out
-
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;
-constexpr uint32_t kSuspendNs = 20000;  // a waiting thread sleeps up to this long per try (hardware wakes it)
-
-// ---- PTX: mbarriers, bulk copies, timer --------------------------------------------------
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{ .reg .pred p;\n"
-        "  mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
-        "  selp.u32 %0, 1, 0, p; }"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(kSuspendNs)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ unsigned long long global_ns() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-// wait for the phase of `parity` to complete; false after the time limit or once
-// another warp of the CTA has given up (then the device error word is set)
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned long long limit_ns = kWaitLimitNs) {
-    if (mbar_test(bar, parity)) return true;
-    const unsigned long long t0 = global_ns();
-    for (;;) {
-        if (mbar_test(bar, parity)) return true;
-        if (*abort_flag || global_ns() - t0 > limit_ns) {
-            *abort_flag = 1;
-            atomicOr(&g_device_error, 1u);
-            return false;
-        }
-    }
-}
-__device__ __forceinline__ unsigned long long l2_policy_keep() {
-    unsigned long long p;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-__device__ __forceinline__ unsigned long long l2_policy_stream() {
-    unsigned long long p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-// global -> shared bulk copy (TMA engine), completion counted on `bar` in bytes
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
-                                          unsigned long long policy) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
-        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar), "l"(policy)
-        : "memory");
-}
-__device__ __forceinline__ float4 lds128(uint32_t addr) {
-    float4 v;
-    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
-    return v;
-}
 
 // ---- consumer work on one stage ----------------------------------------------------------
 //
@@ -219,7 +148,8 @@ __device__ __forceinline__ void block_exp_quant(uint32_t stage, bool valid, floa
 
 template <int F, int CW, int NS>
 __global__ void __launch_bounds__(32 * (CW + 1)) k_exp_quantize_tma(const float* __restrict__ scores, void* codes,
-                                                                  void* scales, long long rows, long long cols) {
+                                                                  void* scales, long long rows, long long cols,
+                                                                  unsigned int* err) {
     constexpr int CH = CW * 4096;  // stage bytes: 32·CW blocks of 128 bytes
     extern __shared__ __align__(128) uint8_t ring[];
     __shared__ __align__(8) unsigned long long full[NS], empty[NS], red[2];
@@ -252,7 +182,7 @@ __global__ void __launch_bounds__(32 * (CW + 1)) k_exp_quantize_tma(const float*
         long long k = 0;
         auto issue = [&](long long i, int j, bool pass_a) -> bool {
             const int s = (int)(k % NS);
-            if (!mbar_wait(smem_u32(&empty[s]), ((uint32_t)(k / NS) & 1u) ^ 1u, ab)) return false;
+            if (!mbar_wait(smem_u32(&empty[s]), ((uint32_t)(k / NS) & 1u) ^ 1u, ab, err)) return false;
             const long long r = blockIdx.x + i * G;
             const uint32_t bytes = (uint32_t)chunk_bytes(j);
             mbar_expect_tx(smem_u32(&full[s]), bytes);
@@ -282,7 +212,7 @@ __global__ void __launch_bounds__(32 * (CW + 1)) k_exp_quantize_tma(const float*
     long long k = 0;
     auto acquire = [&](int& s) -> bool {
         s = (int)(k % NS);
-        const bool ok = mbar_wait(smem_u32(&full[s]), (uint32_t)(k / NS) & 1u, ab);
+        const bool ok = mbar_wait(smem_u32(&full[s]), (uint32_t)(k / NS) & 1u, ab, err);
         return __all_sync(0xFFFFFFFFu, ok);
     };
     auto release = [&](int s) {
@@ -299,7 +229,7 @@ __global__ void __launch_bounds__(32 * (CW + 1)) k_exp_quantize_tma(const float*
             part[p][warp] = acc;
             mbar_arrive(smem_u32(&red[p]));
         }
-        const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&red[p]), (uint32_t)(q >> 1) & 1u, ab));
+        const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&red[p]), (uint32_t)(q >> 1) & 1u, ab, err));
         volatile float* pp = part[p];
         m = pp[0];
 #pragma unroll
@@ -365,7 +295,9 @@ static cudaError_t launch_xt(const float* scores, long long rows, long long cols
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
     long long ctas = (long long)sms * (per_sm > 0 ? per_sm : 1);
     if (ctas > rows) ctas = rows;
-    kern<<<(unsigned)ctas, threads, smem, st>>>(scores, codes, scales, rows, cols);
+    unsigned int* err = nullptr;
+    if ((e = device_error_word(&err)) != cudaSuccess) return e;
+    kern<<<(unsigned)ctas, threads, smem, st>>>(scores, codes, scales, rows, cols, err);
     return cudaGetLastError();
 }
 
@@ -379,7 +311,7 @@ cudaError_t launch_exp_quantize_tma(int fmt, const float* scores, long long rows
 
 // Self-test of the bounded wait: one warp waits on an mbarrier that nothing
 // arrives at; the wait gives up after limit_ns and sets the device error word.
-__global__ void __launch_bounds__(32) k_selftest_timeout(unsigned long long limit_ns) {
+__global__ void __launch_bounds__(32) k_selftest_timeout(unsigned long long limit_ns, unsigned int* err) {
     __shared__ __align__(8) unsigned long long bar;
     __shared__ int abort_flag;
     if (threadIdx.x == 0) {
@@ -388,12 +320,31 @@ __global__ void __launch_bounds__(32) k_selftest_timeout(unsigned long long limi
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
-    mbar_wait(smem_u32(&bar), 0, &abort_flag, limit_ns);
+    mbar_wait(smem_u32(&bar), 0, &abort_flag, err, limit_ns);
 }
 
 cudaError_t launch_selftest_timeout(unsigned long long limit_ns, cudaStream_t st) {
-    k_selftest_timeout<<<1, 32, 0, st>>>(limit_ns);
+    unsigned int* err = nullptr;
+    cudaError_t e = device_error_word(&err);
+    if (e != cudaSuccess) return e;
+    k_selftest_timeout<<<1, 32, 0, st>>>(limit_ns, err);
     return cudaGetLastError();
+}
+
+// address of the device error word on the current device (cached per device)
+cudaError_t device_error_word(unsigned int** p) {
+    static unsigned int* addr[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!addr[dev]) {
+        void* a = nullptr;
+        if ((e = cudaGetSymbolAddress(&a, g_device_error)) != cudaSuccess) return e;
+        addr[dev] = static_cast<unsigned int*>(a);
+    }
+    *p = addr[dev];
+    return cudaSuccess;
 }
 
 cudaError_t read_device_error(unsigned int* value, bool clear) {

@@ -53,6 +53,9 @@ cudaError_t launch_dequantize(int fmt, const void* codes, const void* scales, vo
                               long long nblocks, cudaStream_t st);
 cudaError_t launch_fake_quantize(int fmt, const void* src, void* dst, int dtype, long long nblocks,
                                  cudaStream_t st);
+// the same through the bulk-copy streaming kernel (mxq_stream.cu); 16-byte aligned pointers
+cudaError_t launch_fake_quantize_stream(int fmt, const void* src, void* dst, int dtype, long long nblocks,
+                                        cudaStream_t st);
 // returns cudaErrorNotSupported when cols is beyond what one cluster holds
 cudaError_t launch_exp_quantize(int fmt, const float* scores, long long rows, long long cols, void* codes,
                                 void* scales, cudaStream_t st);
@@ -61,7 +64,9 @@ bool exp_quantize_supported(long long cols);
 bool exp_quantize_tma_supported(int fmt, const void* scores);
 cudaError_t launch_exp_quantize_tma(int fmt, const float* scores, long long rows, long long cols, void* codes,
                                     void* scales, cudaStream_t st);
-// the device error word (bit 0: a bounded wait in a kernel ran out); clear resets it
+// the device error word (bit 0: a bounded wait in a kernel ran out): its device address for
+// kernel arguments, and its value (clear resets it)
+cudaError_t device_error_word(unsigned int** p);
 cudaError_t read_device_error(unsigned int* value, bool clear);
 // one warp waits (bounded by limit_ns) on an mbarrier nothing arrives at
 cudaError_t launch_selftest_timeout(unsigned long long limit_ns, cudaStream_t st);
