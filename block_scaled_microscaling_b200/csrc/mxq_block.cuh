@@ -151,6 +151,28 @@ __device__ __forceinline__ void warp_store6(void* codes, long long first_blk, in
     __syncwarp();
 }
 
+// Inverse of warp_store6: the warp's nvalid 24-byte payloads (consecutive blocks from
+// first_blk) arrive as 16-byte loads shared by the lanes, through shared memory; lane j gets
+// block first_blk + j (lanes past nvalid get stale bytes and must not use them).
+__device__ __forceinline__ void warp_load6(const void* codes, long long first_blk, int nvalid, uint32_t* pw,
+                                           uint8_t* stage, int lane) {
+    const char* g = reinterpret_cast<const char*>(codes) + first_blk * 24;
+    const int nbytes = 24 * nvalid;
+    for (int i = 16 * lane; i + 16 <= nbytes; i += 512) *reinterpret_cast<uint4*>(stage + i) = ld_stream_v4(g + i);
+    if ((nbytes & 15) && lane == 0)
+        *reinterpret_cast<uint2*>(stage + (nbytes & ~15)) = *reinterpret_cast<const uint2*>(g + (nbytes & ~15));
+    __syncwarp();
+    const uint2* q = reinterpret_cast<const uint2*>(stage + 24 * lane);
+    const uint2 a = q[0], b = q[1], c = q[2];
+    pw[0] = a.x;
+    pw[1] = a.y;
+    pw[2] = b.x;
+    pw[3] = b.y;
+    pw[4] = c.x;
+    pw[5] = c.y;
+    __syncwarp();  // the stage is rewritten by the warp's next call
+}
+
 template <int F>
 __device__ __forceinline__ void load_payload(const void* codes, long long b, uint32_t* out, bool a32) {
     const char* p = reinterpret_cast<const char*>(codes) + b * payload<F>();
