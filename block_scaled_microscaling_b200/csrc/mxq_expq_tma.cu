@@ -52,6 +52,14 @@ __device__ unsigned int g_device_error;  // bit 0: a bounded wait ran out
 template <int CW>
 __device__ __forceinline__ float chunk_max(uint32_t stage, int n16, int t) {
     float m = __uint_as_float(0xFF800000u);
+    if (n16 == 256 * CW) {  // a full stage: no bounds checks
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 v = lds128(stage + 16 * (t + 32 * CW * j));
+            m = max3_nan(m, max3_nan(v.x, v.y, v.z), v.w);
+        }
+        return m;
+    }
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int g = t + 32 * CW * j;
@@ -63,49 +71,20 @@ __device__ __forceinline__ float chunk_max(uint32_t stage, int n16, int t) {
     return m;
 }
 
-// 128-bit value (4 words, little-endian) rotated left by 16·k bits, k = 0..7
-__device__ __forceinline__ void rotl128_16(uint32_t (&r)[4], int k) {
-    if (k & 1) {
-        const uint32_t r3 = r[3];
-        r[3] = __funnelshift_l(r[2], r[3], 16);
-        r[2] = __funnelshift_l(r[1], r[2], 16);
-        r[1] = __funnelshift_l(r[0], r[1], 16);
-        r[0] = __funnelshift_l(r3, r[0], 16);
-    }
-    const bool one = k & 2, two = k & 4;
-    uint32_t a0 = one ? r[3] : r[0], a1 = one ? r[0] : r[1], a2 = one ? r[1] : r[2], a3 = one ? r[2] : r[3];
-    r[0] = two ? a2 : a0;
-    r[1] = two ? a3 : a1;
-    r[2] = two ? a0 : a2;
-    r[3] = two ? a1 : a3;
-}
-// 8 words rotated left by k words, k = 0..7
-__device__ __forceinline__ void rotl256_32(uint32_t (&r)[8], int k) {
-#pragma unroll
-    for (int b = 0; b < 3; ++b) {
-        const int sh = 1 << b;
-        const bool on = (k >> b) & 1;
-        uint32_t t[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) t[i] = on ? r[(i - sh + 8) & 7] : r[i];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) r[i] = t[i];
-    }
-}
-
 // pass B: thread t owns block t of the stage. Its 128 bytes are read as eight
-// 16-byte pieces in the order (c + lane) mod 8, so the eight lanes that share a
-// shared-memory wavefront hit eight different bank groups; maximum, exponent
-// and rounding do not depend on the order, and the packed codes are rotated
-// back into place before the store.
+// 16-byte pieces, piece (c xor r) into slot c with r = lane mod 8, so the eight
+// lanes that share a shared-memory wavefront hit eight different bank groups;
+// maximum, exponent and rounding do not depend on the order, and the packed codes
+// are permuted back (slot s holds piece s xor r) before the store.
 template <int F>
 __device__ __forceinline__ void block_exp_quant(uint32_t stage, bool valid, float m, long long b, void* codes,
                                                 void* scales, int t) {
-    const int rot = t & 7;
+    const uint32_t r = (uint32_t)(t & 7);
+    const uint32_t base = (stage + 128u * (uint32_t)t) ^ (16u * r);  // stage + 128 t is 128-byte aligned
     uint32_t w[32];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-        const float4 v = lds128(stage + 128 * t + 16 * ((c + rot) & 7));
+        const float4 v = lds128(base ^ (16u * c));
         w[4 * c] = __float_as_uint(v.x);
         w[4 * c + 1] = __float_as_uint(v.y);
         w[4 * c + 2] = __float_as_uint(v.z);
@@ -122,21 +101,38 @@ __device__ __forceinline__ void block_exp_quant(uint32_t stage, bool valid, floa
     const uint32_t byte = scale_byte<F>(__float_as_uint(pm) & 0x7FFFFFFFu);
     const unsigned long long inv2 = dup2(inv_scale(byte));
     const uint32_t keep = byte == 0xFFu ? 0u : 0xFFFFFFFFu;
-    uint32_t h[8];
+    float a[32];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        float a0, a1, a2, a3;
-        upk(f2mul(pk(__uint_as_float(w[4 * c]), __uint_as_float(w[4 * c + 1])), inv2), a0, a1);
-        upk(f2mul(pk(__uint_as_float(w[4 * c + 2]), __uint_as_float(w[4 * c + 3])), inv2), a2, a3);
-        h[c] = F == F_E2M1 ? (cvt2<F>(a0, a1) | (cvt2<F>(a2, a3) << 8)) : (cvt2<F>(a0, a1) | (cvt2<F>(a2, a3) << 16));
-    }
+    for (int i = 0; i < 16; ++i) upk(f2mul(pk(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1])), inv2), a[2 * i], a[2 * i + 1]);
     if (!valid) return;
     if constexpr (F == F_E2M1) {
-        uint32_t r[4] = {h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16)};
-        rotl128_16(r, rot);
-        st_stream_v4(reinterpret_cast<char*>(codes) + b * 16, make_uint4(r[0] & keep, r[1] & keep, r[2] & keep, r[3] & keep));
+        // word i = codes of slots 2i, 2i+1; output word j = pieces 2j, 2j+1 = word j ^ (r >> 1),
+        // its two halves swapped when r is odd
+        uint32_t h[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            h[i] = __byte_perm(cvt8_e2m1(a[8 * i], a[8 * i + 1], a[8 * i + 2], a[8 * i + 3], a[8 * i + 4], a[8 * i + 5],
+                                         a[8 * i + 6], a[8 * i + 7]),
+                               0, (r & 1) ? 0x1032 : 0x3210);
+        const bool x1 = r & 2, x2 = r & 4;
+        const uint32_t g0 = x1 ? h[1] : h[0], g1 = x1 ? h[0] : h[1], g2 = x1 ? h[3] : h[2], g3 = x1 ? h[2] : h[3];
+        st_stream_v4(reinterpret_cast<char*>(codes) + b * 16,
+                     make_uint4((x2 ? g2 : g0) & keep, (x2 ? g3 : g1) & keep, (x2 ? g0 : g2) & keep, (x2 ? g1 : g3) & keep));
     } else {
-        rotl256_32(h, rot);
+        // word c = codes of slot c; output word j = word j ^ r
+        uint32_t h[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) h[c] = cvt4_e4m3(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
+#pragma unroll
+        for (int bit = 0; bit < 3; ++bit) {
+            const int sh = 1 << bit;
+            const bool on = (r >> bit) & 1;
+            uint32_t u[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) u[j] = on ? h[j ^ sh] : h[j];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) h[j] = u[j];
+        }
         char* p = reinterpret_cast<char*>(codes) + b * 32;
         st_stream_v4(p, make_uint4(h[0] & keep, h[1] & keep, h[2] & keep, h[3] & keep));
         st_stream_v4(p + 16, make_uint4(h[4] & keep, h[5] & keep, h[6] & keep, h[7] & keep));
@@ -147,7 +143,7 @@ __device__ __forceinline__ void block_exp_quant(uint32_t stage, bool valid, floa
 // ---- the kernel ---------------------------------------------------------------------------
 
 template <int F, int CW, int NS>
-__global__ void __launch_bounds__(32 * (CW + 1)) k_exp_quantize_tma(const float* __restrict__ scores, void* codes,
+__global__ void __launch_bounds__(32 * (CW + 1), 1) k_exp_quantize_tma(const float* __restrict__ scores, void* codes,
                                                                   void* scales, long long rows, long long cols,
                                                                   unsigned int* err) {
     constexpr int CH = CW * 4096;  // stage bytes: 32·CW blocks of 128 bytes
