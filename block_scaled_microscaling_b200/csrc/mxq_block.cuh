@@ -70,12 +70,19 @@ __device__ __forceinline__ uint32_t code_pair(const uint32_t* w, int i, float in
     float a, b;
     upk(f2mul(pair<T>(w, i), dup2(inv)), a, b);
     if constexpr (F == F_AXS6) {
-        // sign | min(rne(16|y|), 31), rne by a 1.5*2^23 add; the x16 is exact
-        uint32_t ma = __float_as_uint(fabsf(a) * 16.0f + 12582912.0f) - 0x4B400000u;
-        uint32_t mb = __float_as_uint(fabsf(b) * 16.0f + 12582912.0f) - 0x4B400000u;
-        ma = min(ma, 31u) | ((__float_as_uint(a) >> 26) & 0x20u);
-        mb = min(mb, 31u) | ((__float_as_uint(b) >> 26) & 0x20u);
-        return ma | (mb << 6);
+        // sign | min(rne(16|y|), 31) for both values at once in 16-bit lanes: rne by a
+        // 1.5*2^23 add (the x16 is exact; the sum's low 16 bits are the rounded integer),
+        // the two integers gathered by one byte permute, clamped by one 16x2 minimum; the
+        // signs replicated from the top bytes by a second permute
+        const uint32_t ta = __float_as_uint(fabsf(a) * 16.0f + 12582912.0f);
+        const uint32_t tb = __float_as_uint(fabsf(b) * 16.0f + 12582912.0f);
+        uint32_t m2;
+        asm("min.u16x2 %0, %1, %2;" : "=r"(m2) : "r"(__byte_perm(ta, tb, 0x5410)), "r"(0x001F001Fu));
+        uint32_t sg;  // 0xFFFF / 0 per 16-bit lane: prmt selector nibbles 0xB, 0xF replicate the sign bit of
+                      // byte 3 of a and of b (CUDA's __byte_perm ignores the replicate bit)
+        asm("prmt.b32 %0, %1, %2, 0xFFBB;" : "=r"(sg) : "r"(__float_as_uint(a)), "r"(__float_as_uint(b)));
+        const uint32_t c2 = m2 | (sg & 0x00200020u);
+        return c2 - (c2 >> 16) * 65472u;  // code_a | code_b << 6
     } else if constexpr (Fmt<F>::W == 6) {
         return squeeze6(cvt2<F>(a, b));
     } else {
