@@ -38,7 +38,7 @@ __device__ __forceinline__ void tile_quantize(const BatchOp& op, long long first
     const uint32_t byte = scale_byte<F>(block_amax<T>(w));
     uint32_t out[8];
     encode_block<F, T>(w, byte, out);
-    if constexpr (Fmt<F>::W == 6 && !Fmt<F>::FIXED) {
+    if constexpr (Fmt<F>::W == 6) {
         warp_store6<F>(op.out, first, (int)min(32LL, op.nblocks - first), out, stage, lane);
     } else {
         if (ok) store_payload<F>(op.out, b, out, op.a32);

@@ -48,12 +48,13 @@ __device__ __forceinline__ int find_seg(const SegTable<NSEG>& tab, long long b) 
 // only in the grouped FP6 quantize (decoder layers, ~100M values per launch:
 // 0.92 vs 0.77-0.82 of HBM peak); one block elsewhere (a 47 MB launch loses
 // ~5% with two: fewer, longer threads). Shared-memory staging of 6-bit stores
-// helps single-tensor FP6 quantize (0.91 vs 0.79) but not AXS-6 or grouped.
+// helps single-tensor quantize (MXFP6 0.91 vs 0.79; AXS-6 0.90 vs 0.83 once its
+// rounding was packed into 16-bit lanes) but not the grouped kernel.
 template <int F, typename T, int NSEG> __host__ __device__ constexpr int q_unroll() {
     return (NSEG > 1 && Fmt<F>::W == 6 && !Fmt<F>::FIXED && sizeof(T) == 2) ? 2 : 1;
 }
 template <int F, typename T, int NSEG> __host__ __device__ constexpr bool q_stage() {
-    return NSEG == 1 && Fmt<F>::W == 6 && !Fmt<F>::FIXED;
+    return NSEG == 1 && Fmt<F>::W == 6;
 }
 
 // MMA: scales go to the block-scaled MMA tile layout (single tensor, E8M0 formats); a separate
