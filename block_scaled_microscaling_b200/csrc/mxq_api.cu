@@ -204,8 +204,12 @@ mxq_status mxq_fake_quantize(mxq_format fmt, const void* src, mxq_dtype dtype, i
                              mxq_stream stream) {
     MXQ_TRY(check_fake_args(fmt, src, dtype, rows, cols, dst));
     if (rows == 0) return MXQ_OK;
-    return from_cuda(mxq::launch_fake_quantize_stream((int)fmt, src, dst, (int)dtype, rows * (cols / 32),
-                                                      (cudaStream_t)stream));
+    // the bulk-copy stream pays a pipeline fill and drain that only large tensors amortize (AXS-6 fp32
+    // on B200: 3.0 vs 2.3 us at 8K values, 13.7 vs 13.2 us at 8M, 44.8 vs 50.8 us at 33M values)
+    const long long nb = rows * (cols / 32);
+    if (nb < (1LL << 19))
+        return from_cuda(mxq::launch_fake_quantize((int)fmt, src, dst, (int)dtype, nb, (cudaStream_t)stream));
+    return from_cuda(mxq::launch_fake_quantize_stream((int)fmt, src, dst, (int)dtype, nb, (cudaStream_t)stream));
 }
 
 mxq_status mxq_run_batch(mxq_dtype dtype, const mxq_op* ops, int n, mxq_stream stream) {

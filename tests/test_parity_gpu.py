@@ -153,6 +153,20 @@ def test_fake_quantize_in_place_and_round_trip(fmt):
     assert np.array_equal(bits(host(t)), bits(oracle.fake_quantize(x, fmt)))
 
 
+@pytest.mark.parametrize("fmt", ["axs6", "mxfp6_e3m2", "mxfp4"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_fake_quantize_bulk_copy_stream(fmt, dtype):
+    """Sizes from 2^19 blocks up take the bulk-copy stream kernel: 16411 x 1024 values (525 152
+    blocks, 2052 tiles of 256 with a 32-block tail), out of place and in place."""
+    x = hard_values(16411, 1024, dtype, seed=17)
+    t = dev(x)
+    want = bits(oracle.fake_quantize(x, fmt))
+    out = mxq.fake_quantize(t, fmt)
+    assert np.array_equal(bits(host(out)), want)
+    mxq.fake_quantize(t, fmt, out=t)
+    assert np.array_equal(bits(host(t)), want)
+
+
 def test_outputs_stay_inside_their_buffers():
     """Guard bands: sentinel bytes around every output are untouched."""
     x = hard_values(33, 96, "bf16", seed=3)
