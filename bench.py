@@ -306,43 +306,56 @@ def time_graph(torch, g, replays=1):
 
 
 def e2e_measure(torch, mxq, w_host, steps):
-    """Public API from pinned host memory: H2D weight, one batch launch, D2H every output."""
+    """Public API from pinned host memory, every step: H2D of the weight, one batch launch, D2H of
+    every output. The host->device copy of step k+1 runs on its own stream and overlaps the
+    device->host copies of step k (PCIe is full duplex); two device buffer sets alternate."""
     dev = torch.device("cuda")
     hx = torch.from_numpy(w_host.view(np.int16)).view(torch.bfloat16).pin_memory()
-    x = torch.empty_like(hx, device=dev)
-    outs_h = None
-    st = torch.cuda.current_stream()
+    sets = []
+    for _ in range(2):
+        x = torch.zeros_like(hx, device=dev)
+        ca, sa = mxq.quantize(x, "mxfp6_e2m3")
+        cb, sb = mxq.quantize(x, "mxfp6_e3m2")
+        sets.append({"x": x, "ca": ca, "sa": sa, "cb": cb, "sb": sb, "ya": torch.empty_like(x),
+                     "yb": torch.empty_like(x)})
+    outs_h = [torch.empty_like(sets[0][k], device="cpu").pin_memory() for k in ("ca", "sa", "cb", "sb", "ya", "yb")]
     h2d = hx.numel() * 2
-    d2h = 0
+    d2h = sum(o.numel() * o.element_size() for o in outs_h)
+    s_in, s_work = torch.cuda.Stream(), torch.cuda.Stream()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    done = [None, None]  # event after the batch that last read set p's input
+    torch.cuda.synchronize()
     for it in range(steps + 2):
         if it == 2:
-            torch.cuda.synchronize()
-            t0.record(st)
-        x.copy_(hx, non_blocking=True)
-        if it == 0:  # outputs allocated once: two sets of codes, the dequantize ops read the previous step's
-            ca, sa = mxq.quantize(x, "mxfp6_e2m3")
-            cb, sb = mxq.quantize(x, "mxfp6_e3m2")
-            prev = [t.clone() for t in (ca, sa, cb, sb)]
-            ya, yb = torch.empty_like(x), torch.empty_like(x)
-        else:
-            (ca, sa, cb, sb), prev = prev, [ca, sa, cb, sb]
-        pa, psa, pb, psb = prev
-        mxq.batch([("quantize", "mxfp6_e2m3", x, ca, sa), ("quantize", "mxfp6_e3m2", x, cb, sb),
-                   ("dequantize", "mxfp6_e2m3", pa, psa, ya), ("dequantize", "mxfp6_e3m2", pb, psb, yb)])
-        outs = [ca, sa, cb, sb, ya, yb]
-        if outs_h is None:
-            outs_h = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
-            d2h = sum(o.numel() * o.element_size() for o in outs)
-        for o, h in zip(outs, outs_h):
-            h.copy_(o, non_blocking=True)
-    t1.record(st)
+            s_in.synchronize()
+            s_work.synchronize()
+            t0.record(s_in)
+        p = it % 2
+        cur, prev = sets[p], sets[1 - p]
+        with torch.cuda.stream(s_in):
+            if done[p] is not None:
+                s_in.wait_event(done[p])
+            cur["x"].copy_(hx, non_blocking=True)
+            arrived = torch.cuda.Event()
+            arrived.record(s_in)
+        with torch.cuda.stream(s_work):
+            s_work.wait_event(arrived)
+            mxq.batch([("quantize", "mxfp6_e2m3", cur["x"], cur["ca"], cur["sa"]),
+                       ("quantize", "mxfp6_e3m2", cur["x"], cur["cb"], cur["sb"]),
+                       ("dequantize", "mxfp6_e2m3", prev["ca"], prev["sa"], cur["ya"]),
+                       ("dequantize", "mxfp6_e3m2", prev["cb"], prev["sb"], cur["yb"])])
+            done[p] = torch.cuda.Event()
+            done[p].record(s_work)
+            for k, h in zip(("ca", "sa", "cb", "sb", "ya", "yb"), outs_h):
+                h.copy_(cur[k], non_blocking=True)
+    t1.record(s_work)
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / steps
     step_bytes = 4 * nbytes_q("mxfp6_e2m3", hx.numel(), 2)
     return {"value": round(step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms, 4),
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "overlap": "H2D of step k+1 on its own stream during the D2H of step k"}
 
 
 def time_launches(torch, fns, reps):
