@@ -60,33 +60,51 @@ __device__ __forceinline__ void tile_row_load(const uint8_t* tile, int r, uint32
     }
 }
 
+// Lane j's byte offsets of column j in the swizzled rows, one per swizzle phase (the chunk index
+// is xor-ed with (r / 2) mod 4 for 64-byte rows, r mod 8 for 128-byte rows; within a row-block
+// that phase depends only on the row's index inside the block, so it is a compile-time value
+// in the unrolled loops below and every shared-memory access is a base plus an immediate).
+template <typename T> struct ColOffsets {
+    static constexpr int NP = sizeof(T) == 2 ? 4 : 8;
+    uint32_t off[NP];
+    __device__ __forceinline__ explicit ColOffsets(int j) {
+#pragma unroll
+        for (int q = 0; q < NP; ++q)
+            off[q] = sizeof(T) == 2 ? (uint32_t)(16 * ((j >> 3) ^ q) + 2 * (j & 7)) : (uint32_t)(16 * ((j >> 2) ^ q) + 4 * (j & 3));
+    }
+};
+
 // the 32 values of column j, rows 32*rb .. 32*rb+31, as the words of a block
 // (bf16: two values per word, low half first; fp32: one per word)
 template <typename T>
-__device__ __forceinline__ void gather_column(const uint8_t* tile, int rb, int j, uint32_t* w) {
+__device__ __forceinline__ void gather_column(const uint8_t* tile, int rb, const ColOffsets<T>& co, uint32_t* w) {
     if constexpr (sizeof(T) == 2) {
+        const uint8_t* base = tile + rb * 32 * 64;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const uint32_t lo = *reinterpret_cast<const uint16_t*>(tile + tile_off<T>(32 * rb + 2 * i, j));
-            const uint32_t hi = *reinterpret_cast<const uint16_t*>(tile + tile_off<T>(32 * rb + 2 * i + 1, j));
-            w[i] = lo | (hi << 16);
+        for (int i = 0; i < 16; ++i) {  // rows 2i, 2i + 1: swizzle phase i mod 4
+            const uint32_t lo = *reinterpret_cast<const uint16_t*>(base + (2 * i) * 64 + co.off[i & 3]);
+            const uint32_t hi = *reinterpret_cast<const uint16_t*>(base + (2 * i + 1) * 64 + co.off[i & 3]);
+            w[i] = __byte_perm(lo, hi, 0x5410);
         }
     } else {
+        const uint8_t* base = tile + rb * 32 * 128;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) w[i] = *reinterpret_cast<const uint32_t*>(tile + tile_off<T>(32 * rb + i, j));
+        for (int i = 0; i < 32; ++i) w[i] = *reinterpret_cast<const uint32_t*>(base + i * 128 + co.off[i & 7]);
     }
 }
 template <typename T>
-__device__ __forceinline__ void scatter_column(uint8_t* tile, int rb, int j, const uint32_t* o) {
+__device__ __forceinline__ void scatter_column(uint8_t* tile, int rb, const ColOffsets<T>& co, const uint32_t* o) {
     if constexpr (sizeof(T) == 2) {
+        uint8_t* base = tile + rb * 32 * 64;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            *reinterpret_cast<uint16_t*>(tile + tile_off<T>(32 * rb + 2 * i, j)) = (uint16_t)o[i];
-            *reinterpret_cast<uint16_t*>(tile + tile_off<T>(32 * rb + 2 * i + 1, j)) = (uint16_t)(o[i] >> 16);
+            *reinterpret_cast<uint16_t*>(base + (2 * i) * 64 + co.off[i & 3]) = (uint16_t)o[i];
+            *reinterpret_cast<uint16_t*>(base + (2 * i + 1) * 64 + co.off[i & 3]) = (uint16_t)(o[i] >> 16);
         }
     } else {
+        uint8_t* base = tile + rb * 32 * 128;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) *reinterpret_cast<uint32_t*>(tile + tile_off<T>(32 * rb + i, j)) = o[i];
+        for (int i = 0; i < 32; ++i) *reinterpret_cast<uint32_t*>(base + i * 128 + co.off[i & 7]) = o[i];
     }
 }
 
@@ -97,7 +115,9 @@ __global__ void __launch_bounds__(kColThreads) k_quantize_cols(const void* __res
     constexpr int PB = payload<F>();
     constexpr int SB = Fmt<F>::FIXED ? 2 : 1;
     __shared__ __align__(16) uint8_t tile[kTileRows * kTileCols * sizeof(T)];
-    __shared__ __align__(16) uint8_t out[kTileCols * 8 * PB];
+    constexpr int CS = 8 * PB + 8;  // column stride of the staged payloads: 8 bytes of padding keep the
+                                    // lanes (one column each) on different bank pairs
+    __shared__ __align__(16) uint8_t out[kTileCols * CS];
     __shared__ __align__(16) uint8_t sc[kTileCols * 8 * SB];
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const long long RB = rows / 32;
@@ -116,11 +136,11 @@ __global__ void __launch_bounds__(kColThreads) k_quantize_cols(const void* __res
     __syncthreads();
     if (warp < nrb) {
         uint32_t w[Blk<T>::NW];
-        gather_column<T>(tile, warp, lane, w);
+        gather_column<T>(tile, warp, ColOffsets<T>(lane), w);
         const uint32_t byte = scale_byte<F>(block_amax<T>(w));
         uint32_t o[8];
         encode_block<F, T>(w, byte, o);
-        uint32_t* q = reinterpret_cast<uint32_t*>(out + (lane * 8 + warp) * PB);
+        uint32_t* q = reinterpret_cast<uint32_t*>(out + lane * CS + warp * PB);
 #pragma unroll
         for (int i = 0; i < PB / 4; ++i) q[i] = o[i];
         if constexpr (SB == 2) reinterpret_cast<uint16_t*>(sc)[lane * 8 + warp] = (uint16_t)byte;
@@ -128,11 +148,25 @@ __global__ void __launch_bounds__(kColThreads) k_quantize_cols(const void* __res
     }
     __syncthreads();
     // column j's row-blocks of this chunk are contiguous in the output: nrb * PB bytes
+    if (nrb == 8) {  // full chunk: compile-time strides
+        constexpr int SEG8 = 8 * PB / 8;  // 8-byte pieces per column
+#pragma unroll
+        for (int i = t; i < kTileCols * SEG8; i += kColThreads) {
+            const int j = i / SEG8, k = i % SEG8;
+            const long long g = ((col0 + j) * RB + blockIdx.y * 8) * PB + 8 * k;
+            *reinterpret_cast<uint2*>(reinterpret_cast<char*>(codes) + g) = *reinterpret_cast<const uint2*>(out + j * CS + 8 * k);
+        }
+        const int j = t >> 3, k = t & 7;  // 256 threads = 32 columns x 8 row-blocks
+        const long long g = (col0 + j) * RB + blockIdx.y * 8 + k;
+        if constexpr (SB == 2) reinterpret_cast<uint16_t*>(scales)[g] = reinterpret_cast<const uint16_t*>(sc)[j * 8 + k];
+        else reinterpret_cast<uint8_t*>(scales)[g] = sc[j * 8 + k];
+        return;
+    }
     const int seg = nrb * PB;
     for (int i = t; i < kTileCols * (seg / 8); i += kColThreads) {
         const int j = i / (seg / 8), k = i % (seg / 8);
         const long long g = ((col0 + j) * RB + blockIdx.y * 8) * PB + 8 * k;
-        *reinterpret_cast<uint2*>(reinterpret_cast<char*>(codes) + g) = *reinterpret_cast<const uint2*>(out + j * 8 * PB + 8 * k);
+        *reinterpret_cast<uint2*>(reinterpret_cast<char*>(codes) + g) = *reinterpret_cast<const uint2*>(out + j * CS + 8 * k);
     }
     for (int i = t; i < kTileCols * nrb; i += kColThreads) {
         const int j = i / nrb, k = i % nrb;
@@ -155,14 +189,36 @@ __global__ void __launch_bounds__(kColThreads) k_dequantize_cols(const void* __r
     const int nrows = (int)min((long long)kTileRows, rows - row0);
     const int nrb = nrows / 32;
     const bool a32 = ((reinterpret_cast<uintptr_t>(dst) | (uintptr_t)(cols * sizeof(T))) & 31) == 0;
+    constexpr int SB = Fmt<F>::FIXED ? 2 : 1;
+    constexpr int CS = 8 * PB + 8;  // padded column stride, as in quantize_cols
+    __shared__ __align__(16) uint8_t in[kTileCols * CS];
+    __shared__ __align__(16) uint8_t sc[kTileCols * 8 * SB];
+    // column j's nrb payloads of this chunk are contiguous in the transposed layout: read them
+    // with coalesced 8-byte loads (and the scales with coalesced byte loads) into shared memory
+    {
+        const int seg8 = nrb * PB / 8;
+        for (int i = t; i < kTileCols * seg8; i += kColThreads) {
+            const int j = i / seg8, k = i % seg8;
+            const long long g = ((col0 + j) * RB + blockIdx.y * 8) * PB + 8 * k;
+            *reinterpret_cast<uint2*>(in + j * CS + 8 * k) = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const char*>(codes) + g));
+        }
+        for (int i = t; i < kTileCols * nrb; i += kColThreads) {
+            const int j = i / nrb, k = i % nrb;
+            const long long g = (col0 + j) * RB + blockIdx.y * 8 + k;
+            if constexpr (SB == 2) reinterpret_cast<uint16_t*>(sc)[j * 8 + k] = __ldg(reinterpret_cast<const uint16_t*>(scales) + g);
+            else sc[j * 8 + k] = __ldg(reinterpret_cast<const uint8_t*>(scales) + g);
+        }
+    }
+    __syncthreads();
     if (warp < nrb) {
-        const long long b = (col0 + lane) * RB + blockIdx.y * 8 + warp;  // block of the transposed layout
         uint32_t pw[8];
-        load_payload<F>(codes, b, pw, false);
-        const uint32_t byte = load_scale<F>(scales, b);
+        const uint32_t* q = reinterpret_cast<const uint32_t*>(in + lane * CS + warp * PB);
+#pragma unroll
+        for (int i = 0; i < PB / 4; ++i) pw[i] = q[i];
+        const uint32_t byte = SB == 2 ? (reinterpret_cast<const uint16_t*>(sc)[lane * 8 + warp] & 0xFFu) : sc[lane * 8 + warp];
         uint32_t o[Blk<T>::NW];
         decode_block<F, T>(pw, byte, o);
-        scatter_column<T>(tile, warp, lane, o);
+        scatter_column<T>(tile, warp, ColOffsets<T>(lane), o);
     }
     __syncthreads();
     if (t < nrows) {
