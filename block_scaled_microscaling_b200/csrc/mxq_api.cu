@@ -340,7 +340,7 @@ mxq_status mxq_quantize_exmy(int ebits, int mbits, const void* src, mxq_dtype dt
     MXQ_TRY(check_shape(rows, cols));
     if (rows == 0) return MXQ_OK;
     MXQ_TRY(check_ptr(src, 16));
-    MXQ_TRY(check_ptr(codes, 4));
+    MXQ_TRY(check_ptr(codes, 16));
     MXQ_TRY(check_ptr(scales, 1));
     const size_t W = (size_t)(1 + ebits + mbits), nb = (size_t)rows * (size_t)(cols / 32);
     const size_t nsrc = (size_t)rows * (size_t)cols * dtype_bytes(dtype);
@@ -356,7 +356,7 @@ mxq_status mxq_dequantize_exmy(int ebits, int mbits, const void* codes, const vo
     if (!mxq::exmy_supported(ebits, mbits)) return MXQ_ERR_UNSUPPORTED;
     MXQ_TRY(check_shape(rows, cols));
     if (rows == 0) return MXQ_OK;
-    MXQ_TRY(check_ptr(codes, 4));
+    MXQ_TRY(check_ptr(codes, 16));
     MXQ_TRY(check_ptr(scales, 1));
     MXQ_TRY(check_ptr(dst, 16));
     const size_t W = (size_t)(1 + ebits + mbits), nb = (size_t)rows * (size_t)(cols / 32);

@@ -41,6 +41,9 @@ struct ExmyParams {
     uint32_t sub_lim; // fp32 bits of 2^(1-b): below it the grid step is fixed
     float sub_c;      // 2^(24 - b - M)
     float dec_unit;   // 2^(127 - b)
+    uint32_t emin_b;  // 128 - b: biased fp32 exponent of the smallest normal 2^(1-b)
+    uint32_t cadd;    // ((23 - M) << 23) | 0x400000: the rounding constant's bits less its exponent
+    uint32_t kcode;   // (b - 128) << M (mod 2^32)
 };
 
 static ExmyParams exmy_params(int E, int M) {
@@ -61,16 +64,23 @@ static ExmyParams exmy_params(int E, int M) {
     float df;
     memcpy(&df, &db, 4);
     p.dec_unit = df;
+    p.emin_b = (uint32_t)(128 - b);
+    p.cadd = ((uint32_t)(23 - M) << 23) | 0x400000u;
+    p.kcode = (uint32_t)(b - 128) << M;
     return p;
 }
 
-// magnitude code of y >= 0 (fp32, already scaled)
+// magnitude code of y >= 0 (fp32, already scaled), one formula for the normal and the subnormal
+// range: with e = max(exponent of y, 1 - b), the grid step there is 2^(e - M); adding
+// C = 1.5 * 2^(e + 23 - M) rounds y to that step (round to nearest, ties to even, exact for
+// y / step < 2^22) and leaves q = y / step in the low bits of the sum; the code is
+// (e + b - 1) * 2^M + q (a carry of q into the next binade gives the next binade's first code),
+// clamped to the largest magnitude.
 __device__ __forceinline__ uint32_t exmy_mag(float y, const ExmyParams& p) {
-    const uint32_t u = __float_as_uint(y);
-    const uint32_t r = u + ((1u << (p.shift - 1)) - 1u) + ((u >> p.shift) & 1u);
-    const uint32_t normal = min((r >> p.shift) - p.rebias, p.maxmag);
-    const uint32_t sub = min(__float_as_uint(y + p.sub_c) - __float_as_uint(p.sub_c), p.maxmag);
-    return u < p.sub_lim ? sub : normal;
+    const uint32_t eb = max(__float_as_uint(y) >> 23, p.emin_b);  // biased e
+    const uint32_t cb = eb * 0x800000u + p.cadd;
+    const uint32_t q = __float_as_uint(y + __uint_as_float(cb)) - cb;
+    return min((eb << p.M) + q + p.kcode, p.maxmag);
 }
 
 template <int W> __device__ __forceinline__ void pack_codes(const uint32_t* c, uint32_t* out) {
@@ -133,6 +143,24 @@ __device__ __forceinline__ void exmy_decode(const uint32_t* pw, uint32_t byte, c
     }
 }
 
+// Dequantize: a warp's 32 consecutive payloads (32 x 4W bytes) arrive through shared memory, so
+// that global memory sees 16-byte coalesced loads instead of W 4-byte loads per lane at a 4W-byte
+// stride. stage: 32 * W words of this warp.
+template <int W>
+__device__ __forceinline__ void warp_load_words(const void* codes, long long first_blk, int nvalid, uint32_t* pw,
+                                                uint32_t* stage, int lane) {
+    const char* g = reinterpret_cast<const char*>(codes) + first_blk * 4 * W;
+    const int nbytes = 4 * W * nvalid;
+    for (int i = 16 * lane; i + 16 <= nbytes; i += 512)
+        *reinterpret_cast<uint4*>(reinterpret_cast<char*>(stage) + i) = ld_stream_v4(g + i);
+    if (lane == 0)
+        for (int i = nbytes & ~15; i < nbytes; i += 4) stage[i / 4] = __ldg(reinterpret_cast<const uint32_t*>(g + i));
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < W; ++i) pw[i] = stage[lane * W + i];
+    __syncwarp();
+}
+
 template <int W, typename T>
 __global__ void __launch_bounds__(kExThreads) k_quantize_exmy(const void* __restrict__ src, void* __restrict__ codes,
                                                               uint8_t* __restrict__ scales, long long nblocks,
@@ -145,9 +173,14 @@ __global__ void __launch_bounds__(kExThreads) k_quantize_exmy(const void* __rest
         const uint32_t byte = am >= 0x7F800000u ? 0xFFu : (uint32_t)max((int)(am >> 23) - p.emax, 0);
         uint32_t out[W];
         exmy_encode<W, T>(w, byte, p, out);
-        uint32_t* q = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(codes) + b * 4 * W);
+        char* q = reinterpret_cast<char*>(codes) + b * 4 * W;
+        if constexpr (W == 4 || W == 8) {  // 16 or 32 bytes per lane: whole 16-byte stores
 #pragma unroll
-        for (int i = 0; i < W; ++i) q[i] = out[i];
+            for (int i = 0; i < W; i += 4) st_stream_v4(q + 4 * i, make_uint4(out[i], out[i + 1], out[i + 2], out[i + 3]));
+        } else {
+#pragma unroll
+            for (int i = 0; i < W; ++i) reinterpret_cast<uint32_t*>(q)[i] = out[i];
+        }
         scales[b] = (uint8_t)byte;
     }
 }
@@ -157,16 +190,21 @@ __global__ void __launch_bounds__(kExThreads) k_dequantize_exmy(const void* __re
                                                                 const uint8_t* __restrict__ scales,
                                                                 void* __restrict__ dst, long long nblocks, ExmyParams p,
                                                                 bool a32) {
+    __shared__ __align__(16) uint32_t stage[kExThreads / 32][32 * W];
+    const int lane = threadIdx.x & 31;
     const long long stride = (long long)gridDim.x * kExThreads;
-    for (long long b = (long long)blockIdx.x * kExThreads + threadIdx.x; b < nblocks; b += stride) {
+    for (long long first = (long long)blockIdx.x * kExThreads + (threadIdx.x & ~31); first < nblocks;
+         first += stride) {  // warp-uniform trip count
+        const long long b = first + lane;
+        const int nvalid = (int)min(32LL, nblocks - first);
+        const uint32_t byte = lane < nvalid ? __ldg(scales + b) : 0u;  // in flight with the payloads
         uint32_t pw[W];
-        const uint32_t* q = reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(codes) + b * 4 * W);
-#pragma unroll
-        for (int i = 0; i < W; ++i) pw[i] = __ldg(q + i);
-        const uint32_t byte = __ldg(scales + b);
-        uint32_t o[Blk<T>::NW];
-        exmy_decode<W, T>(pw, byte, p, o);
-        store_block<T>(dst, b, o, a32);
+        warp_load_words<W>(codes, first, nvalid, pw, stage[threadIdx.x >> 5], lane);
+        if (lane < nvalid) {
+            uint32_t o[Blk<T>::NW];
+            exmy_decode<W, T>(pw, byte, p, o);
+            store_block<T>(dst, b, o, a32);
+        }
     }
 }
 

@@ -189,7 +189,7 @@ MXQ_API mxq_status mxq_dequantize_cols(mxq_format fmt, const void* codes, const 
  * (E = 0 is sign + fixed point m/2^(M-1)); no code is reserved for Inf/NaN.
  * Block rule as above with emax = 2^(E-1) (0 for E = 0). Layouts: codes
  * uint8[rows * cols/32 * 4W] (W-bit codes LSB-first, a block's payload is W
- * 32-bit words, 4-byte aligned), scales uint8[rows * cols/32] E8M0 bytes.
+ * 32-bit words; the array 16-byte aligned), scales uint8[rows * cols/32] E8M0 bytes.
  * e2m1 / e2m3 / e3m2 give exactly MXFP4 / MXFP6 E2M3 / E3M2; e0m5 gives AXS-6's
  * codes (with a one-byte scale). Rounding is integer arithmetic on the fp32
  * bit patterns (no conversion instruction exists for arbitrary splits).
