@@ -4,14 +4,17 @@
 // codes [cols, rows/32 * P] and scales [cols, rows/32], so a consumer reads
 // each column's blocks contiguously.
 //
-// Tile: 256 rows x 32 columns. Loads: one thread per row, the row's 64 (bf16)
-// or 128 (fp32) bytes as whole 32-byte sectors, into shared memory with 16-byte
-// chunks permuted per row (conflict-free writes). Compute: warp w takes
-// row-block w, lane j column j; all lanes read the same row at once (a
-// permutation of one row: conflict-free). Payloads are staged per column and
-// leave as contiguous runs of the column's row-blocks.
+// Tile: 256 rows x 128 bytes (64 bf16 or 32 fp32 columns; the last strip of a
+// bf16 matrix may be 32 columns wide). Loads: one thread per row, the row's
+// bytes as whole 32-byte sectors, into shared memory with the 16-byte chunk c
+// of row r at chunk index c ^ (r mod 8) (conflict-free writes). Compute: warp w
+// takes row-block w, lane l the CPL = 128 / (32 * sizeof(T)) columns l*CPL ..;
+// for a row, the 32 lanes read one 4-byte word each (all 128 bytes of the row:
+// conflict-free), and for bf16 a byte permute splits each word into the two
+// columns. Payloads and scales are staged per column (in the tile's memory,
+// once its values are in registers) and leave as contiguous runs of the
+// column's row-blocks.
 #include <cstdint>
-#include <mutex>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -23,11 +26,164 @@ namespace mxq {
 
 constexpr int kColThreads = 256;
 constexpr int kTileRows = 256;  // 8 row-blocks
-constexpr int kTileCols = 32;
+constexpr int kRowBytes = 128;  // bytes of a tile row
+
+template <typename T> struct ColTile {
+    static constexpr int TC = kRowBytes / (int)sizeof(T);  // columns per tile
+    static constexpr int CPL = TC / 32;                     // columns per lane
+};
+
+// byte offset of 4-byte word q (0..31) of tile row r
+__device__ __forceinline__ uint32_t word_off(int r, int q) {
+    return (uint32_t)(r * kRowBytes + 16 * ((q >> 2) ^ (r & 7)) + 4 * (q & 3));
+}
+
+// row r of the tile from / to registers, 16 bytes per chunk, the first nch chunks
+__device__ __forceinline__ void tile_row_store(uint8_t* tile, int r, const uint32_t* w, int nch) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        if (c < nch)
+            *reinterpret_cast<uint4*>(tile + r * kRowBytes + 16 * (c ^ (r & 7))) =
+                make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+}
+__device__ __forceinline__ void tile_row_load(const uint8_t* tile, int r, uint32_t* w, int nch) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        if (c < nch) {
+            const uint4 v = *reinterpret_cast<const uint4*>(tile + r * kRowBytes + 16 * (c ^ (r & 7)));
+            w[4 * c] = v.x;
+            w[4 * c + 1] = v.y;
+            w[4 * c + 2] = v.z;
+            w[4 * c + 3] = v.w;
+        }
+}
+
+// The CPL blocks of lane `lane`'s columns in row-block rb: block k holds column lane*CPL + k,
+// as the words of a block (bf16: two values per word, low half first; fp32: one per word).
+// Within a row-block the swizzle phase r mod 8 is a compile-time value in the unrolled loops.
+template <typename T>
+__device__ __forceinline__ void gather_columns(const uint8_t* tile, int rb, int lane, uint32_t (*w)[Blk<T>::NW]) {
+    const uint8_t* base = tile + rb * 32 * kRowBytes;
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {  // rows 2i, 2i + 1: columns 2 lane, 2 lane + 1 share a word
+            const uint32_t a = *reinterpret_cast<const uint32_t*>(base + word_off(2 * i, lane));
+            const uint32_t b = *reinterpret_cast<const uint32_t*>(base + word_off(2 * i + 1, lane));
+            w[0][i] = __byte_perm(a, b, 0x5410);
+            w[1][i] = __byte_perm(a, b, 0x7632);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) w[0][i] = *reinterpret_cast<const uint32_t*>(base + word_off(i, lane));
+    }
+}
+template <typename T>
+__device__ __forceinline__ void scatter_columns(uint8_t* tile, int rb, int lane, const uint32_t (*o)[Blk<T>::NW]) {
+    uint8_t* base = tile + rb * 32 * kRowBytes;
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            *reinterpret_cast<uint32_t*>(base + word_off(2 * i, lane)) = __byte_perm(o[0][i], o[1][i], 0x5410);
+            *reinterpret_cast<uint32_t*>(base + word_off(2 * i + 1, lane)) = __byte_perm(o[0][i], o[1][i], 0x7632);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) *reinterpret_cast<uint32_t*>(base + word_off(i, lane)) = o[0][i];
+    }
+}
+
+// grid: (column strips of TC, row chunks of 256); rows % 32 == 0, cols % 32 == 0
+template <int F, typename T>
+__global__ void __launch_bounds__(kColThreads) k_quantize_cols(const void* __restrict__ src, void* __restrict__ codes,
+                                                              void* __restrict__ scales, long long rows, long long cols) {
+    constexpr int TC = ColTile<T>::TC, CPL = ColTile<T>::CPL;
+    constexpr int PB = payload<F>();
+    constexpr int SB = Fmt<F>::FIXED ? 2 : 1;
+    constexpr int CS = 8 * PB + 8;  // column stride of the staged payloads: 8 bytes of padding keep the
+                                    // lanes (one column each) on different bank pairs
+    static_assert(TC * CS + TC * 8 * SB <= kTileRows * kRowBytes, "staging fits in the tile");
+    __shared__ __align__(16) uint8_t tile[kTileRows * kRowBytes];
+    uint8_t* const out = tile;                // staged payloads and scales reuse the tile once
+    uint8_t* const sc = tile + TC * CS;       // every warp has gathered its columns
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const long long RB = rows / 32;
+    const long long col0 = (long long)blockIdx.x * TC;
+    const long long row0 = (long long)blockIdx.y * kTileRows;
+    const int nrows = (int)min((long long)kTileRows, rows - row0);
+    const int nrb = nrows / 32;
+    const int ncols = (int)min((long long)TC, cols - col0);
+    const int rowbytes = ncols * (int)sizeof(T);  // 64 or 128
+    const bool a32 = ((reinterpret_cast<uintptr_t>(src) | (uintptr_t)(cols * sizeof(T))) & 31) == 0;
+    if (t < nrows) {
+        uint32_t w[32];
+        const char* p = reinterpret_cast<const char*>(src) + ((row0 + t) * cols + col0) * (long long)sizeof(T);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (32 * i < rowbytes) ld32(p + 32 * i, w + 8 * i, a32);
+        tile_row_store(tile, t, w, rowbytes / 16);
+    }
+    __syncthreads();
+    uint32_t w[CPL][Blk<T>::NW];
+    if (warp < nrb) gather_columns<T>(tile, warp, lane, w);
+    __syncthreads();  // the tile's bytes are in registers: its memory takes the staged outputs
+    if (warp < nrb) {
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) {
+            const int j = lane * CPL + k;  // column within the strip
+            if (j < ncols) {
+                const uint32_t byte = scale_byte<F>(block_amax<T>(w[k]));
+                uint32_t o[8];
+                encode_block<F, T>(w[k], byte, o);
+                uint32_t* q = reinterpret_cast<uint32_t*>(out + j * CS + warp * PB);
+#pragma unroll
+                for (int i = 0; i < PB / 4; ++i) q[i] = o[i];
+                if constexpr (SB == 2) reinterpret_cast<uint16_t*>(sc)[j * 8 + warp] = (uint16_t)byte;
+                else sc[j * 8 + warp] = (uint8_t)byte;
+            }
+        }
+    }
+    __syncthreads();
+    // column j's row-blocks of this chunk are contiguous in the output: nrb * PB bytes
+    if (nrb == 8 && ncols == TC) {  // full tile: compile-time strides
+        constexpr int SEG8 = PB;    // 8-byte pieces per column (8 row-blocks x PB bytes / 8)
+#pragma unroll
+        for (int i = t; i < TC * SEG8; i += kColThreads) {
+            const int j = i / SEG8, k = i % SEG8;
+            const long long g = ((col0 + j) * RB + blockIdx.y * 8) * PB + 8 * k;
+            *reinterpret_cast<uint2*>(reinterpret_cast<char*>(codes) + g) = *reinterpret_cast<const uint2*>(out + j * CS + 8 * k);
+        }
+#pragma unroll
+        for (int i = t; i < TC * 8; i += kColThreads) {
+            const int j = i >> 3, k = i & 7;
+            const long long g = (col0 + j) * RB + blockIdx.y * 8 + k;
+            if constexpr (SB == 2) reinterpret_cast<uint16_t*>(scales)[g] = reinterpret_cast<const uint16_t*>(sc)[j * 8 + k];
+            else reinterpret_cast<uint8_t*>(scales)[g] = sc[j * 8 + k];
+        }
+        return;
+    }
+    const int seg8 = nrb * PB / 8;
+    for (int i = t; i < ncols * seg8; i += kColThreads) {
+        const int j = i / seg8, k = i % seg8;
+        const long long g = ((col0 + j) * RB + blockIdx.y * 8) * PB + 8 * k;
+        *reinterpret_cast<uint2*>(reinterpret_cast<char*>(codes) + g) = *reinterpret_cast<const uint2*>(out + j * CS + 8 * k);
+    }
+    for (int i = t; i < ncols * nrb; i += kColThreads) {
+        const int j = i / nrb, k = i % nrb;
+        const long long g = (col0 + j) * RB + blockIdx.y * 8 + k;
+        if constexpr (SB == 2) reinterpret_cast<uint16_t*>(scales)[g] = reinterpret_cast<const uint16_t*>(sc)[j * 8 + k];
+        else reinterpret_cast<uint8_t*>(scales)[g] = sc[j * 8 + k];
+    }
+}
+
+// ---- dequantize: 32-column tiles (64-byte bf16 rows) -------------------------------------------
+// The 128-byte-row tile above was slower for dequantize (bf16 16384x8192: 0.53 vs 0.62 of the
+// HBM peak), so dequantize keeps tiles of 256 rows x 32 columns, chunk c of row r at c ^ (r/2 mod 4)
+// for 64-byte rows and c ^ (r mod 8) for 128-byte rows.
+constexpr int kNarrowCols = 32;
 
 // byte offset of element (r, j) of the tile; rows of 32 * sizeof(T) bytes,
 // chunk c of row r stored at c ^ sw(r)
-template <typename T> __device__ __forceinline__ uint32_t tile_off(int r, int j) {
+template <typename T> __device__ __forceinline__ uint32_t ntile_off(int r, int j) {
     if constexpr (sizeof(T) == 2) {
         const int c = j >> 3;  // 4 chunks of 8 values
         return (uint32_t)(r * 64 + 16 * (c ^ ((r >> 1) & 3)) + 2 * (j & 7));
@@ -38,16 +194,7 @@ template <typename T> __device__ __forceinline__ uint32_t tile_off(int r, int j)
 }
 
 template <typename T>
-__device__ __forceinline__ void tile_row_store(uint8_t* tile, int r, const uint32_t* w) {
-    constexpr int NC = sizeof(T) == 2 ? 4 : 8;
-#pragma unroll
-    for (int c = 0; c < NC; ++c) {
-        const int pos = sizeof(T) == 2 ? (c ^ ((r >> 1) & 3)) : (c ^ (r & 7));
-        *reinterpret_cast<uint4*>(tile + r * 16 * NC + 16 * pos) = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-    }
-}
-template <typename T>
-__device__ __forceinline__ void tile_row_load(const uint8_t* tile, int r, uint32_t* w) {
+__device__ __forceinline__ void ntile_row_load(const uint8_t* tile, int r, uint32_t* w) {
     constexpr int NC = sizeof(T) == 2 ? 4 : 8;
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
@@ -64,36 +211,18 @@ __device__ __forceinline__ void tile_row_load(const uint8_t* tile, int r, uint32
 // is xor-ed with (r / 2) mod 4 for 64-byte rows, r mod 8 for 128-byte rows; within a row-block
 // that phase depends only on the row's index inside the block, so it is a compile-time value
 // in the unrolled loops below and every shared-memory access is a base plus an immediate).
-template <typename T> struct ColOffsets {
+template <typename T> struct NColOffsets {
     static constexpr int NP = sizeof(T) == 2 ? 4 : 8;
     uint32_t off[NP];
-    __device__ __forceinline__ explicit ColOffsets(int j) {
+    __device__ __forceinline__ explicit NColOffsets(int j) {
 #pragma unroll
         for (int q = 0; q < NP; ++q)
             off[q] = sizeof(T) == 2 ? (uint32_t)(16 * ((j >> 3) ^ q) + 2 * (j & 7)) : (uint32_t)(16 * ((j >> 2) ^ q) + 4 * (j & 3));
     }
 };
 
-// the 32 values of column j, rows 32*rb .. 32*rb+31, as the words of a block
-// (bf16: two values per word, low half first; fp32: one per word)
 template <typename T>
-__device__ __forceinline__ void gather_column(const uint8_t* tile, int rb, const ColOffsets<T>& co, uint32_t* w) {
-    if constexpr (sizeof(T) == 2) {
-        const uint8_t* base = tile + rb * 32 * 64;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {  // rows 2i, 2i + 1: swizzle phase i mod 4
-            const uint32_t lo = *reinterpret_cast<const uint16_t*>(base + (2 * i) * 64 + co.off[i & 3]);
-            const uint32_t hi = *reinterpret_cast<const uint16_t*>(base + (2 * i + 1) * 64 + co.off[i & 3]);
-            w[i] = __byte_perm(lo, hi, 0x5410);
-        }
-    } else {
-        const uint8_t* base = tile + rb * 32 * 128;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) w[i] = *reinterpret_cast<const uint32_t*>(base + i * 128 + co.off[i & 7]);
-    }
-}
-template <typename T>
-__device__ __forceinline__ void scatter_column(uint8_t* tile, int rb, const ColOffsets<T>& co, const uint32_t* o) {
+__device__ __forceinline__ void nscatter_column(uint8_t* tile, int rb, const NColOffsets<T>& co, const uint32_t* o) {
     if constexpr (sizeof(T) == 2) {
         uint8_t* base = tile + rb * 32 * 64;
 #pragma unroll
@@ -108,101 +237,34 @@ __device__ __forceinline__ void scatter_column(uint8_t* tile, int rb, const ColO
     }
 }
 
-// grid: (column strips, row chunks); rows % 32 == 0, cols % 32 == 0
-template <int F, typename T>
-__global__ void __launch_bounds__(kColThreads) k_quantize_cols(const void* __restrict__ src, void* __restrict__ codes,
-                                                              void* __restrict__ scales, long long rows, long long cols) {
-    constexpr int PB = payload<F>();
-    constexpr int SB = Fmt<F>::FIXED ? 2 : 1;
-    __shared__ __align__(16) uint8_t tile[kTileRows * kTileCols * sizeof(T)];
-    constexpr int CS = 8 * PB + 8;  // column stride of the staged payloads: 8 bytes of padding keep the
-                                    // lanes (one column each) on different bank pairs
-    __shared__ __align__(16) uint8_t out[kTileCols * CS];
-    __shared__ __align__(16) uint8_t sc[kTileCols * 8 * SB];
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const long long RB = rows / 32;
-    const long long col0 = (long long)blockIdx.x * kTileCols;
-    const long long row0 = (long long)blockIdx.y * kTileRows;
-    const int nrows = (int)min((long long)kTileRows, rows - row0);
-    const int nrb = nrows / 32;
-    const bool a32 = ((reinterpret_cast<uintptr_t>(src) | (uintptr_t)(cols * sizeof(T))) & 31) == 0;
-    if (t < nrows) {
-        uint32_t w[8 * sizeof(T)];
-        const char* p = reinterpret_cast<const char*>(src) + ((row0 + t) * cols + col0) * (long long)sizeof(T);
-#pragma unroll
-        for (int i = 0; i < (int)sizeof(T); ++i) ld32(p + 32 * i, w + 8 * i, a32);  // 32 * sizeof(T) bytes
-        tile_row_store<T>(tile, t, w);
-    }
-    __syncthreads();
-    if (warp < nrb) {
-        uint32_t w[Blk<T>::NW];
-        gather_column<T>(tile, warp, ColOffsets<T>(lane), w);
-        const uint32_t byte = scale_byte<F>(block_amax<T>(w));
-        uint32_t o[8];
-        encode_block<F, T>(w, byte, o);
-        uint32_t* q = reinterpret_cast<uint32_t*>(out + lane * CS + warp * PB);
-#pragma unroll
-        for (int i = 0; i < PB / 4; ++i) q[i] = o[i];
-        if constexpr (SB == 2) reinterpret_cast<uint16_t*>(sc)[lane * 8 + warp] = (uint16_t)byte;
-        else sc[lane * 8 + warp] = (uint8_t)byte;
-    }
-    __syncthreads();
-    // column j's row-blocks of this chunk are contiguous in the output: nrb * PB bytes
-    if (nrb == 8) {  // full chunk: compile-time strides
-        constexpr int SEG8 = 8 * PB / 8;  // 8-byte pieces per column
-#pragma unroll
-        for (int i = t; i < kTileCols * SEG8; i += kColThreads) {
-            const int j = i / SEG8, k = i % SEG8;
-            const long long g = ((col0 + j) * RB + blockIdx.y * 8) * PB + 8 * k;
-            *reinterpret_cast<uint2*>(reinterpret_cast<char*>(codes) + g) = *reinterpret_cast<const uint2*>(out + j * CS + 8 * k);
-        }
-        const int j = t >> 3, k = t & 7;  // 256 threads = 32 columns x 8 row-blocks
-        const long long g = (col0 + j) * RB + blockIdx.y * 8 + k;
-        if constexpr (SB == 2) reinterpret_cast<uint16_t*>(scales)[g] = reinterpret_cast<const uint16_t*>(sc)[j * 8 + k];
-        else reinterpret_cast<uint8_t*>(scales)[g] = sc[j * 8 + k];
-        return;
-    }
-    const int seg = nrb * PB;
-    for (int i = t; i < kTileCols * (seg / 8); i += kColThreads) {
-        const int j = i / (seg / 8), k = i % (seg / 8);
-        const long long g = ((col0 + j) * RB + blockIdx.y * 8) * PB + 8 * k;
-        *reinterpret_cast<uint2*>(reinterpret_cast<char*>(codes) + g) = *reinterpret_cast<const uint2*>(out + j * CS + 8 * k);
-    }
-    for (int i = t; i < kTileCols * nrb; i += kColThreads) {
-        const int j = i / nrb, k = i % nrb;
-        const long long g = (col0 + j) * RB + blockIdx.y * 8 + k;
-        if constexpr (SB == 2) reinterpret_cast<uint16_t*>(scales)[g] = reinterpret_cast<const uint16_t*>(sc)[j * 8 + k];
-        else reinterpret_cast<uint8_t*>(scales)[g] = sc[j * 8 + k];
-    }
-}
 
 template <int F, typename T>
 __global__ void __launch_bounds__(kColThreads) k_dequantize_cols(const void* __restrict__ codes,
                                                                 const void* __restrict__ scales, void* __restrict__ dst,
                                                                 long long rows, long long cols) {
     constexpr int PB = payload<F>();
-    __shared__ __align__(16) uint8_t tile[kTileRows * kTileCols * sizeof(T)];
+    __shared__ __align__(16) uint8_t tile[kTileRows * kNarrowCols * sizeof(T)];
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const long long RB = rows / 32;
-    const long long col0 = (long long)blockIdx.x * kTileCols;
+    const long long col0 = (long long)blockIdx.x * kNarrowCols;
     const long long row0 = (long long)blockIdx.y * kTileRows;
     const int nrows = (int)min((long long)kTileRows, rows - row0);
     const int nrb = nrows / 32;
     const bool a32 = ((reinterpret_cast<uintptr_t>(dst) | (uintptr_t)(cols * sizeof(T))) & 31) == 0;
     constexpr int SB = Fmt<F>::FIXED ? 2 : 1;
     constexpr int CS = 8 * PB + 8;  // padded column stride, as in quantize_cols
-    __shared__ __align__(16) uint8_t in[kTileCols * CS];
-    __shared__ __align__(16) uint8_t sc[kTileCols * 8 * SB];
+    __shared__ __align__(16) uint8_t in[kNarrowCols * CS];
+    __shared__ __align__(16) uint8_t sc[kNarrowCols * 8 * SB];
     // column j's nrb payloads of this chunk are contiguous in the transposed layout: read them
     // with coalesced 8-byte loads (and the scales with coalesced byte loads) into shared memory
     {
         const int seg8 = nrb * PB / 8;
-        for (int i = t; i < kTileCols * seg8; i += kColThreads) {
+        for (int i = t; i < kNarrowCols * seg8; i += kColThreads) {
             const int j = i / seg8, k = i % seg8;
             const long long g = ((col0 + j) * RB + blockIdx.y * 8) * PB + 8 * k;
             *reinterpret_cast<uint2*>(in + j * CS + 8 * k) = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const char*>(codes) + g));
         }
-        for (int i = t; i < kTileCols * nrb; i += kColThreads) {
+        for (int i = t; i < kNarrowCols * nrb; i += kColThreads) {
             const int j = i / nrb, k = i % nrb;
             const long long g = (col0 + j) * RB + blockIdx.y * 8 + k;
             if constexpr (SB == 2) reinterpret_cast<uint16_t*>(sc)[j * 8 + k] = __ldg(reinterpret_cast<const uint16_t*>(scales) + g);
@@ -218,12 +280,12 @@ __global__ void __launch_bounds__(kColThreads) k_dequantize_cols(const void* __r
         const uint32_t byte = SB == 2 ? (reinterpret_cast<const uint16_t*>(sc)[lane * 8 + warp] & 0xFFu) : sc[lane * 8 + warp];
         uint32_t o[Blk<T>::NW];
         decode_block<F, T>(pw, byte, o);
-        scatter_column<T>(tile, warp, ColOffsets<T>(lane), o);
+        nscatter_column<T>(tile, warp, NColOffsets<T>(lane), o);
     }
     __syncthreads();
     if (t < nrows) {
         uint32_t w[8 * sizeof(T)];
-        tile_row_load<T>(tile, t, w);
+        ntile_row_load<T>(tile, t, w);
         char* p = reinterpret_cast<char*>(dst) + ((row0 + t) * cols + col0) * (long long)sizeof(T);
 #pragma unroll
         for (int i = 0; i < (int)sizeof(T); ++i) st32(p + 32 * i, w + 8 * i, a32);
@@ -233,20 +295,21 @@ __global__ void __launch_bounds__(kColThreads) k_dequantize_cols(const void* __r
 template <int F, typename T>
 static cudaError_t launch_qc_t(const void* src, void* codes, void* scales, long long rows, long long cols,
                                cudaStream_t st) {
-    dim3 grid((unsigned)(cols / kTileCols), (unsigned)((rows + kTileRows - 1) / kTileRows));
+    constexpr int TC = ColTile<T>::TC;
+    dim3 grid((unsigned)((cols + TC - 1) / TC), (unsigned)((rows + kTileRows - 1) / kTileRows));
     k_quantize_cols<F, T><<<grid, kColThreads, 0, st>>>(src, codes, scales, rows, cols);
     return cudaGetLastError();
 }
 template <int F, typename T>
 static cudaError_t launch_dqc_t(const void* codes, const void* scales, void* dst, long long rows, long long cols,
                                 cudaStream_t st) {
-    dim3 grid((unsigned)(cols / kTileCols), (unsigned)((rows + kTileRows - 1) / kTileRows));
+    dim3 grid((unsigned)(cols / kNarrowCols), (unsigned)((rows + kTileRows - 1) / kTileRows));
     k_dequantize_cols<F, T><<<grid, kColThreads, 0, st>>>(codes, scales, dst, rows, cols);
     return cudaGetLastError();
 }
 
 bool cols_grid_ok(long long rows, long long cols) {
-    return cols / kTileCols <= 0x7FFFFFFFLL && (rows + kTileRows - 1) / kTileRows <= 65535;
+    return (cols + 31) / 32 <= 0x7FFFFFFFLL && (rows + kTileRows - 1) / kTileRows <= 65535;
 }
 
 cudaError_t launch_quantize_cols(int fmt, const void* src, int dtype, long long rows, long long cols, void* codes,
