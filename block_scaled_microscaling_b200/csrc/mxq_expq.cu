@@ -24,24 +24,6 @@
 
 namespace mxq {
 
-
-template <int F>
-__device__ __forceinline__ void exp_quant_block(uint32_t (&w)[32], float mr, long long blk, void* codes, void* scales,
-                                                bool a32) {
-    exp_values<32>(w, mr);
-    float q[11];
-#pragma unroll
-    for (int i = 0; i < 10; ++i) q[i] = max3_nan(__uint_as_float(w[3 * i]), __uint_as_float(w[3 * i + 1]), __uint_as_float(w[3 * i + 2]));
-    q[10] = max_nan(__uint_as_float(w[30]), __uint_as_float(w[31]));
-    float pm = max3_nan(max3_nan(q[0], q[1], q[2]), max3_nan(q[3], q[4], q[5]), max3_nan(q[6], q[7], q[8]));
-    pm = max3_nan(pm, q[9], q[10]);  // p >= 0 or NaN: the block maximum (or NaN)
-    const uint32_t byte = scale_byte<F>(__float_as_uint(pm) & 0x7FFFFFFFu);
-    uint32_t out[8];
-    encode_block<F, float>(w, byte, out);
-    store_payload<F>(codes, blk, out, a32);
-    store_scale<F>(scales, blk, byte);
-}
-
 __device__ __forceinline__ float max32(const uint32_t (&w)[32]) {
     float m[11];
 #pragma unroll

@@ -8,23 +8,24 @@
 // maximum must be complete before the first exponential, so a row is read
 // twice: pass A for its maximum, pass B for exp + quantize.
 //
-// One persistent CTA per SM; a producer thread streams 64 KB stages of scores
-// (4 KB per consumer warp) into a ring of three shared-memory stages with
-// cp.async.bulk (the TMA engine), each stage guarded by a "full" and an "empty"
-// mbarrier; sixteen consumer warps read the stages. The producer's order
-// interleaves pass B of row i with pass A of row i+1 stage by stage, so HBM
-// streams the next row while the current one is exponentiated; pass A's copies
-// ask L2 to keep the row (evict_last), pass B's copies find it there
-// (evict_first), and HBM sees each score once. The row maximum is combined
-// across the consumer warps through a shared-memory slot and an mbarrier
-// (double-buffered by row parity). Any row length: a row is a sequence of
-// stages, the last one partial.
-//
-// Pass A: each consumer thread takes eight 16-byte pieces of the stage
-// (conflict-free: a warp reads 512 consecutive bytes). Pass B: a thread owns a
-// block of 32 keys (block_exp_quant: read in a lane-rotated order so that the
-// shared-memory wavefronts are conflict-free, codes rotated back before the
-// store).
+// One persistent CTA per SM walks its rows (row blockIdx.x + i * gridDim.x) with
+// three warp roles:
+//  - a producer thread streams every row, in order, through a ring of 32 KB
+//    shared-memory stages with cp.async.bulk (the TMA engine), each stage guarded
+//    by a "full" and an "empty" mbarrier; the copies ask L2 to keep the row
+//    (evict_last). Before the first stage of row i it waits until the consumers
+//    have finished row i - LEAD, which bounds the rows a CTA holds in L2;
+//  - MW maximum warps take each stage as soon as it lands, fold it into the row
+//    maximum and free it, so the ring refills at once and HBM always has the
+//    whole ring in flight; at the end of a row they combine their partial maxima
+//    and publish the row maximum in one of four slots (mbarrier "mready");
+//  - CW consumer warps (pass B): for row i they wait for its maximum, then each
+//    thread reads blocks of 32 scores straight from L2 with 32-byte loads (marked
+//    evict_first: last use), exponentiates and quantizes them in registers and
+//    stores codes and scales; then they signal "bfree" for the row.
+// HBM therefore reads each score once, and the HBM stream never waits for the
+// exponentials of earlier rows except through the LEAD bound. Any row length: a
+// row is a sequence of stages, the last one partial.
 //
 // Every wait is bounded (one second by %globaltimer, or sooner once another
 // warp has given up): a wait that runs out sets the library's device error
@@ -43,26 +44,24 @@ namespace mxq {
 
 __device__ unsigned int g_device_error;  // bit 0: a bounded wait ran out
 
-// ---- consumer work on one stage ----------------------------------------------------------
-//
-// A stage holds 32·CW blocks of 32 scores (CW consumer warps, 4 KB per warp).
+constexpr int kXStageBytes = 32768;  // one ring stage: 256 blocks of 32 scores
 
-// pass A: maximum of the stage's first n16 16-byte pieces (NaN if any is NaN);
-// piece g = t + 32·CW·j, so a warp reads 512 consecutive bytes per load
-template <int CW>
-__device__ __forceinline__ float chunk_max(uint32_t stage, int n16, int t) {
+// maximum of the stage's first n16 16-byte pieces (NaN if any is NaN); thread t of
+// the NT maximum threads takes pieces t + NT·j, so a warp reads 512 consecutive bytes
+template <int NT>
+__device__ __forceinline__ float stage_max(uint32_t stage, int n16, int t) {
+    constexpr int PER = kXStageBytes / 16 / NT;
     float m = __uint_as_float(0xFF800000u);
-    if (n16 == 256 * CW) {  // a full stage: no bounds checks
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float4 v = lds128(stage + 16 * (t + 32 * CW * j));
+    if (n16 == kXStageBytes / 16) {  // a full stage: no bounds checks
+#pragma unroll 8
+        for (int j = 0; j < PER; ++j) {
+            const float4 v = lds128(stage + 16 * (t + NT * j));
             m = max3_nan(m, max3_nan(v.x, v.y, v.z), v.w);
         }
         return m;
     }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const int g = t + 32 * CW * j;
+    for (int j = 0; j < PER; ++j) {
+        const int g = t + NT * j;
         if (g < n16) {
             const float4 v = lds128(stage + 16 * g);
             m = max3_nan(m, max3_nan(v.x, v.y, v.z), v.w);
@@ -71,85 +70,21 @@ __device__ __forceinline__ float chunk_max(uint32_t stage, int n16, int t) {
     return m;
 }
 
-// pass B: thread t owns block t of the stage. Its 128 bytes are read as eight
-// 16-byte pieces, piece (c xor r) into slot c with r = lane mod 8, so the eight
-// lanes that share a shared-memory wavefront hit eight different bank groups;
-// maximum, exponent and rounding do not depend on the order, and the packed codes
-// are permuted back (slot s holds piece s xor r) before the store.
-template <int F>
-__device__ __forceinline__ void block_exp_quant(uint32_t stage, bool valid, float m, long long b, void* codes,
-                                                void* scales, int t) {
-    const uint32_t r = (uint32_t)(t & 7);
-    const uint32_t base = (stage + 128u * (uint32_t)t) ^ (16u * r);  // stage + 128 t is 128-byte aligned
-    uint32_t w[32];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const float4 v = lds128(base ^ (16u * c));
-        w[4 * c] = __float_as_uint(v.x);
-        w[4 * c + 1] = __float_as_uint(v.y);
-        w[4 * c + 2] = __float_as_uint(v.z);
-        w[4 * c + 3] = __float_as_uint(v.w);
-    }
-    exp_values<32>(w, m);
-    float q[11];
-#pragma unroll
-    for (int i = 0; i < 10; ++i)
-        q[i] = max3_nan(__uint_as_float(w[3 * i]), __uint_as_float(w[3 * i + 1]), __uint_as_float(w[3 * i + 2]));
-    q[10] = max_nan(__uint_as_float(w[30]), __uint_as_float(w[31]));
-    float pm = max3_nan(max3_nan(q[0], q[1], q[2]), max3_nan(q[3], q[4], q[5]), max3_nan(q[6], q[7], q[8]));
-    pm = max3_nan(pm, q[9], q[10]);  // p >= 0 or NaN
-    const uint32_t byte = scale_byte<F>(__float_as_uint(pm) & 0x7FFFFFFFu);
-    const unsigned long long inv2 = dup2(inv_scale(byte));
-    const uint32_t keep = byte == 0xFFu ? 0u : 0xFFFFFFFFu;
-    float a[32];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) upk(f2mul(pk(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1])), inv2), a[2 * i], a[2 * i + 1]);
-    if (!valid) return;
-    if constexpr (F == F_E2M1) {
-        // word i = codes of slots 2i, 2i+1; output word j = pieces 2j, 2j+1 = word j ^ (r >> 1),
-        // its two halves swapped when r is odd
-        uint32_t h[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            h[i] = __byte_perm(cvt8_e2m1(a[8 * i], a[8 * i + 1], a[8 * i + 2], a[8 * i + 3], a[8 * i + 4], a[8 * i + 5],
-                                         a[8 * i + 6], a[8 * i + 7]),
-                               0, (r & 1) ? 0x1032 : 0x3210);
-        const bool x1 = r & 2, x2 = r & 4;
-        const uint32_t g0 = x1 ? h[1] : h[0], g1 = x1 ? h[0] : h[1], g2 = x1 ? h[3] : h[2], g3 = x1 ? h[2] : h[3];
-        st_stream_v4(reinterpret_cast<char*>(codes) + b * 16,
-                     make_uint4((x2 ? g2 : g0) & keep, (x2 ? g3 : g1) & keep, (x2 ? g0 : g2) & keep, (x2 ? g1 : g3) & keep));
-    } else {
-        // word c = codes of slot c; output word j = word j ^ r
-        uint32_t h[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) h[c] = cvt4_e4m3(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
-#pragma unroll
-        for (int bit = 0; bit < 3; ++bit) {
-            const int sh = 1 << bit;
-            const bool on = (r >> bit) & 1;
-            uint32_t u[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) u[j] = on ? h[j ^ sh] : h[j];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) h[j] = u[j];
-        }
-        char* p = reinterpret_cast<char*>(codes) + b * 32;
-        st_stream_v4(p, make_uint4(h[0] & keep, h[1] & keep, h[2] & keep, h[3] & keep));
-        st_stream_v4(p + 16, make_uint4(h[4] & keep, h[5] & keep, h[6] & keep, h[7] & keep));
-    }
-    reinterpret_cast<uint8_t*>(scales)[b] = (uint8_t)byte;
+__device__ __forceinline__ void named_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 // ---- the kernel ---------------------------------------------------------------------------
 
-template <int F, int CW, int NS>
-__global__ void __launch_bounds__(32 * (CW + 1), 1) k_exp_quantize_tma(const float* __restrict__ scores, void* codes,
-                                                                  void* scales, long long rows, long long cols,
-                                                                  unsigned int* err) {
-    constexpr int CH = CW * 4096;  // stage bytes: 32·CW blocks of 128 bytes
+template <int F, int CW, int MW, int NS, int LEAD>
+__global__ void __launch_bounds__(32 * (CW + MW + 1), 1)
+    k_exp_quantize_tma(const float* __restrict__ scores, void* codes, void* scales, long long rows, long long cols,
+                       bool a32, unsigned int* err) {
+    static_assert(LEAD >= 1 && LEAD <= 4, "four row slots bound the producer's lead");
+    constexpr int CH = kXStageBytes, NM = 32 * MW;
     extern __shared__ __align__(128) uint8_t ring[];
-    __shared__ __align__(8) unsigned long long full[NS], empty[NS], red[2];
-    __shared__ float part[2][CW];
+    __shared__ __align__(8) unsigned long long full[NS], empty[NS], mready[4], bfree[4];
+    __shared__ float mval[4], mpart[2][MW];
     __shared__ int abort_flag;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const long long G = gridDim.x;
@@ -159,10 +94,12 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1) k_exp_quantize_tma(const flo
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(smem_u32(&full[s]), 1);
-            mbar_init(smem_u32(&empty[s]), CW);
+            mbar_init(smem_u32(&empty[s]), MW);
         }
-        mbar_init(smem_u32(&red[0]), CW);
-        mbar_init(smem_u32(&red[1]), CW);
+        for (int s = 0; s < 4; ++s) {
+            mbar_init(smem_u32(&mready[s]), 1);
+            mbar_init(smem_u32(&bfree[s]), CW);
+        }
         abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -172,26 +109,26 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1) k_exp_quantize_tma(const flo
     const uint32_t ring0 = smem_u32(ring);
     auto chunk_bytes = [&](int j) { return (int)min((long long)CH, rowbytes - (long long)j * CH); };
 
-    if (warp == CW) {  // producer: one thread issues every copy
+    if (warp == CW + MW) {  // producer: one thread issues every copy
         if (lane != 0) return;
-        const unsigned long long keep = l2_policy_keep(), strm = l2_policy_stream();
+        const unsigned long long keep = l2_policy_keep();
         long long k = 0;
-        auto issue = [&](long long i, int j, bool pass_a) -> bool {
-            const int s = (int)(k % NS);
-            if (!mbar_wait(smem_u32(&empty[s]), ((uint32_t)(k / NS) & 1u) ^ 1u, ab, err)) return false;
-            const long long r = blockIdx.x + i * G;
-            const uint32_t bytes = (uint32_t)chunk_bytes(j);
-            mbar_expect_tx(smem_u32(&full[s]), bytes);
-            bulk_load(ring0 + s * CH, reinterpret_cast<const char*>(scores) + r * rowbytes + (long long)j * CH, bytes,
-                      smem_u32(&full[s]), pass_a ? keep : strm);
-            ++k;
-            return true;
-        };
         bool ok = true;
-        for (int j = 0; j < nc && ok; ++j) ok = issue(0, j, true);
-        for (long long i = 0; i + 1 < n && ok; ++i)
-            for (int j = 0; j < nc && ok; ++j) ok = issue(i, j, false) && issue(i + 1, j, true);
-        for (int j = 0; j < nc && ok; ++j) ok = issue(n - 1, j, false);
+        for (long long i = 0; i < n && ok; ++i) {
+            if (i >= LEAD) {  // the consumers are done with row i - LEAD
+                const long long q = i - LEAD;
+                ok = mbar_wait(smem_u32(&bfree[q & 3]), (uint32_t)(q >> 2) & 1u, ab, err);
+            }
+            const char* src = reinterpret_cast<const char*>(scores) + (blockIdx.x + i * G) * rowbytes;
+            for (int j = 0; j < nc && ok; ++j, ++k) {
+                const int s = (int)(k % NS);
+                ok = mbar_wait(smem_u32(&empty[s]), ((uint32_t)(k / NS) & 1u) ^ 1u, ab, err);
+                if (!ok) break;
+                const uint32_t bytes = (uint32_t)chunk_bytes(j);
+                mbar_expect_tx(smem_u32(&full[s]), bytes);
+                bulk_load(ring0 + s * CH, src + (long long)j * CH, bytes, smem_u32(&full[s]), keep);
+            }
+        }
         if (!ok) {
             // gave up: let the copies still in flight land before the CTA's shared memory goes away
             for (long long q = k > NS ? k - NS : 0; q < k; ++q) {
@@ -204,85 +141,76 @@ __global__ void __launch_bounds__(32 * (CW + 1), 1) k_exp_quantize_tma(const flo
         return;
     }
 
-    // consumers: tid 0 .. 32·CW - 1
-    long long k = 0;
-    auto acquire = [&](int& s) -> bool {
-        s = (int)(k % NS);
-        const bool ok = mbar_wait(smem_u32(&full[s]), (uint32_t)(k / NS) & 1u, ab, err);
-        return __all_sync(0xFFFFFFFFu, ok);
-    };
-    auto release = [&](int s) {
+    if (warp >= CW) {  // maximum warps: pass A
+        const int t = tid - 32 * CW, mw = warp - CW;
+        long long k = 0;
+        const float NEG_INF = __uint_as_float(0xFF800000u);
+        for (long long i = 0; i < n; ++i) {
+            float acc = NEG_INF;
+            for (int j = 0; j < nc; ++j, ++k) {
+                const int s = (int)(k % NS);
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&full[s]), (uint32_t)(k / NS) & 1u, ab, err))) return;
+                acc = max_nan(acc, stage_max<NM>(ring0 + s * CH, chunk_bytes(j) / 16, t));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc = max_nan(acc, __shfl_xor_sync(0xFFFFFFFFu, acc, o));
+            const int p = (int)(i & 1);
+            if (lane == 0) mpart[p][mw] = acc;
+            if constexpr (MW > 1) named_sync(1, NM);
+            else __syncwarp();
+            if (t == 0) {
+                float m = mpart[p][0];
+#pragma unroll
+                for (int w = 1; w < MW; ++w) m = max_nan(m, mpart[p][w]);
+                mval[i & 3] = m;
+                mbar_arrive(smem_u32(&mready[i & 3]));  // release: mval is visible to the waiters
+            }
+        }
+        return;
+    }
+
+    // consumers: pass B, thread tid of 32·CW
+    const char* sc = reinterpret_cast<const char*>(scores);
+    for (long long i = 0; i < n; ++i) {
+        const int slot = (int)(i & 3);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&mready[slot]), (uint32_t)(i >> 2) & 1u, ab, err))) return;
+        const float m = *reinterpret_cast<volatile float*>(&mval[slot]);
+        const long long row = blockIdx.x + i * G;
+        const char* s = sc + row * rowbytes;
+        for (long long b = tid; b < bpr; b += 32 * CW) {
+            uint32_t w[32];
+            load_block<float>(s, b, w, a32);
+            exp_quant_block<F>(w, m, row * bpr + b, codes, scales, a32);
+        }
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
-        ++k;
-    };
-    // row maximum over the consumer warps; q = this CTA's row counter (slot q & 1)
-    auto reduce = [&](float acc, long long q, float& m) -> bool {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc = max_nan(acc, __shfl_xor_sync(0xFFFFFFFFu, acc, o));
-        const int p = (int)(q & 1);
-        if (lane == 0) {
-            part[p][warp] = acc;
-            mbar_arrive(smem_u32(&red[p]));
-        }
-        const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&red[p]), (uint32_t)(q >> 1) & 1u, ab, err));
-        volatile float* pp = part[p];
-        m = pp[0];
-#pragma unroll
-        for (int w = 1; w < CW; ++w) m = max_nan(m, pp[w]);
-        return ok;
-    };
-    const float NEG_INF = __uint_as_float(0xFF800000u);
-    float acc = NEG_INF, mB = 0.0f;
-    int s;
-    for (int j = 0; j < nc; ++j) {  // pass A of the first row
-        if (!acquire(s)) return;
-        acc = max_nan(acc, chunk_max<CW>(ring0 + s * CH, chunk_bytes(j) / 16, tid));
-        release(s);
-    }
-    if (!reduce(acc, 0, mB)) return;
-    for (long long i = 0; i + 1 < n; ++i) {  // pass B of row i, pass A of row i + 1, stage by stage
-        const long long blk_row = (blockIdx.x + i * G) * bpr;
-        acc = NEG_INF;
-        for (int j = 0; j < nc; ++j) {
-            if (!acquire(s)) return;
-            block_exp_quant<F>(ring0 + s * CH, tid < chunk_bytes(j) / 128, mB, blk_row + (long long)j * 32 * CW + tid,
-                               codes, scales, tid);
-            release(s);
-            if (!acquire(s)) return;
-            acc = max_nan(acc, chunk_max<CW>(ring0 + s * CH, chunk_bytes(j) / 16, tid));
-            release(s);
-        }
-        if (!reduce(acc, i + 1, mB)) return;
-    }
-    const long long blk_row = (blockIdx.x + (n - 1) * G) * bpr;
-    for (int j = 0; j < nc; ++j) {  // pass B of the last row
-        if (!acquire(s)) return;
-        block_exp_quant<F>(ring0 + s * CH, tid < chunk_bytes(j) / 128, mB, blk_row + (long long)j * 32 * CW + tid,
-                           codes, scales, tid);
-        release(s);
+        if (lane == 0) mbar_arrive(smem_u32(&bfree[slot]));
     }
 }
 
 // ---- launch -----------------------------------------------------------------------------
 
-// Shape by measurement on B200 (fp32 4096 x 32768 scores -> MXFP4, fraction of the copy peak):
-// 16 consumer warps and three 64 KB stages, one CTA per SM: 0.72; 8 warps x 3 x 32 KB, two CTAs
-// per SM: 0.72; 8 warps x 6 x 32 KB, one CTA: 0.62; 4 warps x 3 x 16 KB, four CTAs: 0.70. An L2
-// prefetch of the row after next did not help (0.70). Keeping the row resident in shared memory
-// and freeing it in pass B, so that each score crosses L2 -> SM once, was slower (0.54): the
-// next row cannot stream in while the current one fills two thirds of the ring.
-constexpr int kXWarps = 16, kXStages = 3;
+// Shape by measurement on B200 (fp32 4096 x 32768 scores -> MXFP4, fraction of the copy peak;
+// consumer warps / maximum warps / stages / lead): 16/2/4/3 0.82-0.83 (kept); 16/2/6/2 0.72,
+// 16/2/6/3 0.81, 16/2/6/4 0.82, 16/4/6/3 0.81, 16/4/4/3 0.82, 16/1/6/2 0.63, 12/2/6/3 0.76,
+// 20/2/4/3 0.79, 24/2/4/3 0.78. A lead of two rows starves the HBM stream: the producer's
+// ring runs more than a row ahead of the landed data, so it reaches the row gate while
+// the consumers still wait for the row the gate names. Two blocks in flight per consumer
+// thread (0.81) and an L1 prefetch of a thread's next block (0.79) did not help. The
+// previous design, one ring shared by both passes with the passes interleaved stage by
+// stage, reached 0.76: at most one HBM stage per SM was in flight.
+constexpr int kXWarps = 16, kXMaxWarps = 2, kXStages = 4, kXLead = 3;
 
 bool exp_quantize_tma_supported(int fmt, const void* scores) {
     return (fmt == F_E2M1 || fmt == F_E4M3) && (reinterpret_cast<uintptr_t>(scores) & 15) == 0;
 }
 
-template <int F, int CW, int NS>
+template <int F, int CW, int MW, int NS, int LEAD>
 static cudaError_t launch_xt(const float* scores, long long rows, long long cols, void* codes, void* scales,
                              cudaStream_t st) {
-    auto kern = k_exp_quantize_tma<F, CW, NS>;
-    const int smem = NS * CW * 4096, threads = 32 * (CW + 1);
+    auto kern = k_exp_quantize_tma<F, CW, MW, NS, LEAD>;
+    const int smem = NS * kXStageBytes, threads = 32 * (CW + MW + 1);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148, per_sm = 1;
@@ -293,15 +221,16 @@ static cudaError_t launch_xt(const float* scores, long long rows, long long cols
     if (ctas > rows) ctas = rows;
     unsigned int* err = nullptr;
     if ((e = device_error_word(&err)) != cudaSuccess) return e;
-    kern<<<(unsigned)ctas, threads, smem, st>>>(scores, codes, scales, rows, cols, err);
+    const bool a32 = ((reinterpret_cast<uintptr_t>(scores) | reinterpret_cast<uintptr_t>(codes)) & 31) == 0;
+    kern<<<(unsigned)ctas, threads, smem, st>>>(scores, codes, scales, rows, cols, a32, err);
     return cudaGetLastError();
 }
 
 cudaError_t launch_exp_quantize_tma(int fmt, const float* scores, long long rows, long long cols, void* codes,
                                     void* scales, cudaStream_t st) {
     if (rows == 0) return cudaSuccess;
-    if (fmt == F_E2M1) return launch_xt<F_E2M1, kXWarps, kXStages>(scores, rows, cols, codes, scales, st);
-    if (fmt == F_E4M3) return launch_xt<F_E4M3, kXWarps, kXStages>(scores, rows, cols, codes, scales, st);
+    if (fmt == F_E2M1) return launch_xt<F_E2M1, kXWarps, kXMaxWarps, kXStages, kXLead>(scores, rows, cols, codes, scales, st);
+    if (fmt == F_E4M3) return launch_xt<F_E4M3, kXWarps, kXMaxWarps, kXStages, kXLead>(scores, rows, cols, codes, scales, st);
     return cudaErrorInvalidValue;
 }
 

@@ -251,9 +251,9 @@ def test_grouped_matches_oracle(fmt):
 @pytest.mark.parametrize("fmt", ["mxfp4", "mxfp8", "mxfp6_e2m3", "axs6"])
 @pytest.mark.parametrize("rows,cols", [(3000, 640), (700, 8192), (5, 131072), (3, 262144 + 32), (149, 4128)])
 def test_exp_quantize_many_rows_per_cta(fmt, rows, cols):
-    """More rows than resident CTAs: each CTA walks several rows (for MXFP4/MXFP8 through the
-    bulk-copy ring, pass B of one row interleaved with pass A of the next; rows of one full
-    chunk plus a partial one)."""
+    """More rows than resident CTAs: each CTA walks several rows (for MXFP4/MXFP8 the row
+    stream runs up to three rows ahead of pass B, so the row-slot rings wrap many times; rows of
+    one full stage plus a partial one, rows shorter than one stage)."""
     s = synthetic.attention_scores(seed=5, heads=1, queries=rows, keys=cols)
     s[::97, 3] = np.nan
     s[1::89, :] = -np.inf
