@@ -207,14 +207,27 @@ int resident_ctas(const void* fn, int dev) {
     return ctas;
 }
 
+// Two grid shapes, chosen per kernel by measurement on B200 (graphs of back-to-back launches
+// on HBM-resident data, fraction of the copy peak):
+//  - persistent (one_pass = false): SMs x resident CTAs, each thread walks its blocks
+//    grid-stride, U at a time;
+//  - one pass (one_pass = true): one CTA per 256 blocks, each thread one block; the hardware
+//    starts a new CTA wherever one finishes.
+// Single-tensor quantize takes one pass at every size (bf16 16384x8192: MXFP6 0.90 -> 0.97,
+// MXFP8 0.93 -> 1.04; bf16 4096x4096: 0.76 -> 0.78), and so do dequantize with per-thread
+// payload loads above 2^21 blocks (MXFP8 16384x8192: 0.89 -> 1.01). Persistent stays where
+// it measured better: the grouped quantize with two blocks in flight (decoder layer 0.92 vs
+// 0.87), the batch kernel (0.91 vs 0.88), dequantize at 47 MB (E2M3 0.90 vs 0.87) and the
+// warp-shared 6-bit dequantize (0.94 vs 0.88).
 template <typename K>
-static int grid_for(K kernel, long long nblocks) {
+static int grid_for(K kernel, long long nblocks, bool one_pass = false) {
+    long long want = (nblocks + kThreads - 1) / kThreads;
+    if (want < 1) want = 1;
+    if (one_pass) return (int)(want < 0x7FFFFFFFLL ? want : 0x7FFFFFFFLL);
     int dev = 0;
     cudaGetDevice(&dev);
-    long long cap = resident_ctas(reinterpret_cast<const void*>(kernel), dev);
-    // fill every SM first; a thread then takes its blocks U at a time
-    long long want = (nblocks + kThreads - 1) / kThreads;
-    return (int)(want < cap ? (want > 0 ? want : 1) : cap);
+    const long long cap = resident_ctas(reinterpret_cast<const void*>(kernel), dev);
+    return (int)(want < cap ? want : cap);
 }
 
 static bool aligned32(const void* a, const void* b) {
@@ -229,7 +242,7 @@ static cudaError_t launch_q(const SegTable<NSEG>& tab, cudaStream_t st) {
     } else {
         if (tab.seg[0].kb_mma) return cudaErrorInvalidValue;
     }
-    k<<<grid_for(k, tab.nblocks), kThreads, 0, st>>>(tab);
+    k<<<grid_for(k, tab.nblocks, NSEG == 1), kThreads, 0, st>>>(tab);
     return cudaGetLastError();
 }
 
@@ -262,9 +275,10 @@ template cudaError_t launch_quantize<kMaxSeg>(int, int, SegTable<kMaxSeg>&, cuda
 template <int F, typename T>
 static cudaError_t launch_dq_t(const void* codes, const void* scales, void* dst, long long nb, cudaStream_t st) {
     auto k = k_dequantize<F, T>;
-    if constexpr (Fmt<F>::W == 6)
-        if (nb >= (1LL << 21)) k = k_dequantize<F, T, true>;  // >= 64M values
-    k<<<grid_for(k, nb), kThreads, 0, st>>>(codes, scales, dst, nb, aligned32(codes, dst));
+    bool coop = false;
+    if constexpr (Fmt<F>::W == 6) coop = nb >= (1LL << 21);  // >= 64M values
+    if (coop) k = k_dequantize<F, T, Fmt<F>::W == 6>;
+    k<<<grid_for(k, nb, !coop && nb >= (1LL << 21)), kThreads, 0, st>>>(codes, scales, dst, nb, aligned32(codes, dst));
     return cudaGetLastError();
 }
 

@@ -224,13 +224,21 @@ __global__ void __launch_bounds__(kExThreads) k_fake_quantize_exmy(const void* s
     }
 }
 
-static int ex_grid(const void* fn, long long nb) {
+// Grid: one CTA per 256 blocks (one pass: the hardware starts a CTA wherever one finishes) for
+// dequantize and fake-quantize, SMs x resident CTAs walking grid-stride for quantize. Measured
+// on bf16 16384x8192 over five splits (fraction of the copy peak): dequantize 0.85-0.94 ->
+// 0.90-0.93, fake-quantize 0.67-0.70 -> 0.70-0.72 with one pass; quantize, bound by its integer
+// rounding, 0.62-0.74 persistent vs 0.62-0.68 in one pass.
+static int ex_grid(const void* fn, long long nb, bool one_pass) {
+    long long want = (nb + kExThreads - 1) / kExThreads;
+    if (want < 1) want = 1;
+    if (one_pass) return (int)(want < 0x7FFFFFFFLL ? want : 0x7FFFFFFFLL);
     int dev = 0, sms = 148, per = 1;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, kExThreads, 0);
-    long long cap = (long long)sms * (per > 0 ? per : 1), want = (nb + kExThreads - 1) / kExThreads;
-    return (int)(want < cap ? (want > 0 ? want : 1) : cap);
+    const long long cap = (long long)sms * (per > 0 ? per : 1);
+    return (int)(want < cap ? want : cap);
 }
 static bool al32(const void* a, const void* b) {
     return ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b)) & 31) == 0;
@@ -241,15 +249,15 @@ static cudaError_t ex_launch(int op, const void* in, void* out, const void* aux_
                              const ExmyParams& p, cudaStream_t st) {
     if (op == 0) {
         auto k = k_quantize_exmy<W, T>;
-        k<<<ex_grid((const void*)k, nb), kExThreads, 0, st>>>(in, out, reinterpret_cast<uint8_t*>(aux_out), nb, p,
+        k<<<ex_grid((const void*)k, nb, false), kExThreads, 0, st>>>(in, out, reinterpret_cast<uint8_t*>(aux_out), nb, p,
                                                             al32(in, in));
     } else if (op == 1) {
         auto k = k_dequantize_exmy<W, T>;
-        k<<<ex_grid((const void*)k, nb), kExThreads, 0, st>>>(in, reinterpret_cast<const uint8_t*>(aux_in), out, nb, p,
+        k<<<ex_grid((const void*)k, nb, true), kExThreads, 0, st>>>(in, reinterpret_cast<const uint8_t*>(aux_in), out, nb, p,
                                                             al32(out, out));
     } else {
         auto k = k_fake_quantize_exmy<W, T>;
-        k<<<ex_grid((const void*)k, nb), kExThreads, 0, st>>>(in, out, nb, p, al32(in, out));
+        k<<<ex_grid((const void*)k, nb, true), kExThreads, 0, st>>>(in, out, nb, p, al32(in, out));
     }
     return cudaGetLastError();
 }
