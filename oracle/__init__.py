@@ -46,6 +46,7 @@ def lib():
         L.orc_exp_quantize.argtypes = [i32, vp, i64, i64, vp, vp]
         L.orc_expf.restype = ctypes.c_float
         L.orc_expf.argtypes = [ctypes.c_float]
+        L.orc_exp_free_quantize.argtypes = [vp, i64, i64, vp, vp]
         L.orc_codes_bytes.restype = i64
         L.orc_codes_bytes.argtypes = [i32, i64, i64]
         L.orc_scales_bytes.restype = i64
@@ -172,6 +173,20 @@ def exp_quantize(scores, fmt="mxfp4"):
     rc = lib().orc_exp_quantize(FORMATS[fmt], _ptr(s), rows, cols, _ptr(codes), _ptr(scales))
     if rc:
         raise ValueError(f"oracle exp_quantize rejected the arguments (rc={rc})")
+    return codes, scales
+
+
+def exp_free_quantize(scores):
+    """scores: [rows, cols] float32 -> (codes, scales) of the exp-free E2M1 rule: per block of 32
+    shifted scores an exponent-only scale from the block's maximum of u = (s - rowmax)/ln 2 and
+    code = clamp(rint(2u - 2Es) + 2, 0, 7) (see oracle.c; constants are a reading of the page)."""
+    s = np.ascontiguousarray(scores, dtype=np.float32)
+    rows, cols = s.shape
+    codes = np.zeros((rows, cols // 32 * payload_bytes("mxfp4")), dtype=np.uint8)
+    scales = np.zeros((rows, cols // 32), dtype=np.uint8)
+    rc = lib().orc_exp_free_quantize(_ptr(s), rows, cols, _ptr(codes), _ptr(scales))
+    if rc:
+        raise ValueError(f"oracle exp_free_quantize rejected the arguments (rc={rc})")
     return codes, scales
 
 

@@ -502,6 +502,80 @@ int orc_exp_quantize(int f, const float* scores, int64_t rows, int64_t cols,
     return 0;
 }
 
+/* ---- exp-free E2M1 probabilities (EFQ-Softmax) ------------------------ */
+/*
+ * [EFQ] opening paragraph, "What is it" and the paragraph on the per-block
+ * rule: instead of exponentiating the shifted scores and quantizing the
+ * result, each microscaling block takes an exponent-only scale from its own
+ * local maximum, normalizes the shifted scores with it and maps them to
+ * nonnegative E2M1 codes with one affine rule; no exponential is evaluated.
+ * The page gives neither the slope nor the offset of that rule. Reading
+ * adopted (PARITY UNPINNED against the paper's constants, which are not on
+ * the page; the rule below is pinned to exp-then-quantize where the two must
+ * agree):
+ *   d     = RN(s - m)                  shifted score, fp32, m = row maximum
+ *   u     = RN(d * L2E)                log2 of the probability exp(d), fp32
+ *   u_max = max over the block's 32 u  (NaN if any is NaN)
+ *   Es    = clamp(floor(u_max) - 2, -127, 127)    exponent-only block scale
+ *           (2 = floor(log2 6), E2M1's emax, as for the named formats);
+ *           byte Es + 127; a NaN block stores 0xFF and codes 0
+ *   w     = RN(2*u - 2*Es)             one fused multiply-add, fp32
+ *   code  = clamp(rint(w) + 2, 0, 7)   ties to even; sign bit 0
+ * The E2M1 magnitudes 1, 2, 4 (codes 2, 4, 6) sit at log2 0, 1, 2 and the
+ * odd codes 1.5, 3, 6 at log2 0.58, 1.58, 2.58, so code = 2*log2(p/2^Es) + 2
+ * is the straight line through the grid in the log domain: exact at every
+ * even code and within 0.17 of a code step at the odd ones. Its decoded
+ * value E2M1(code) * 2^Es approximates exp(d).
+ */
+int orc_exp_free_quantize(const float* scores, int64_t rows, int64_t cols, uint8_t* codes, uint8_t* scales) {
+    const float L2E = 0x1.715476p+0f;
+    if (rows < 0 || cols <= 0 || cols % 32) return 2;
+    int64_t bpr = cols / 32;
+    float u[32];
+    uint32_t c[32];
+    for (int64_t r = 0; r < rows; ++r) {
+        const float* s = scores + r * cols;
+        float m = -INFINITY;
+        int has_nan = 0;
+        for (int64_t j = 0; j < cols; ++j) {
+            if (isnan(s[j])) has_nan = 1;
+            else if (s[j] > m) m = s[j];
+        }
+        if (has_nan) m = NAN;
+        for (int64_t bj = 0; bj < bpr; ++bj) {
+            float umax = -INFINITY;
+            int nan_block = 0;
+            for (int i = 0; i < 32; ++i) {
+                float d = s[32 * bj + i] - m;   /* fp32 subtraction */
+                u[i] = d * L2E;                 /* fp32 product */
+                if (isnan(u[i])) nan_block = 1;
+                else if (u[i] > umax) umax = u[i];
+            }
+            int64_t b = r * bpr + bj;
+            int byte;
+            if (nan_block) {
+                byte = 0xFF;
+                for (int i = 0; i < 32; ++i) c[i] = 0;
+            } else {
+                double fl = floor((double)umax);
+                int es = fl < -200.0 ? -127 : (int)fl - 2;
+                if (es < -127) es = -127;
+                if (es > 127) es = 127;
+                byte = es + 127;
+                for (int i = 0; i < 32; ++i) {
+                    float w = fmaf(2.0f, u[i], -2.0f * (float)es);
+                    double k = isinf(w) ? (w < 0 ? -1e9 : 1e9) : (double)rintf(w);
+                    k += 2.0;
+                    c[i] = k < 0.0 ? 0u : (k > 7.0 ? 7u : (uint32_t)k);
+                }
+            }
+            pack_block(&FMT[ORC_E2M1], c, codes + b * payload_bytes(&FMT[ORC_E2M1]));
+            scales[b] = (uint8_t)byte;
+        }
+    }
+    return 0;
+}
+
 /* sizes, for the test harness */
 int64_t orc_codes_bytes(int f, int64_t rows, int64_t cols) {
     return fmt_ok(f) ? rows * (cols / 32) * payload_bytes(&FMT[f]) : -1;
