@@ -435,15 +435,19 @@ def workloads_breakdown(torch, mxq, hbm):
     gen.manual_seed(4)
     sc = torch.randn(4096, 32768, device=dev, generator=gen) * 3
     c5, s5 = mxq.exp_quantize(sc, "mxfp4")
-    ts = time_launches(torch, [lambda: mxq.exp_quantize(sc, "mxfp4", codes=c5, scales=s5)], 10)
+    ts = time_launches(torch, [lambda: mxq.exp_quantize(sc, "mxfp4", codes=c5, scales=s5),
+                               lambda: mxq.exp_free_quantize(sc, codes=c5, scales=s5)], 10)
     rec("c5_scores_exp_mxfp4_f32", nbytes_q("mxfp4", sc.numel(), 4), sc.numel(), ts[0])
+    # the same stage by the exp-free rule (no exponential), same bytes
+    rec("c5_scores_exp_free_mxfp4_f32", nbytes_q("mxfp4", sc.numel(), 4), sc.numel(), ts[1])
     del sc, c5, s5
     torch.cuda.empty_cache()
     return out
 
 
 PROFILE_CASES = ["batch_weight", "q_e2m3_weight", "q_e3m2_weight", "dq_e2m3_weight", "q_mxfp8_act", "dq_mxfp8_act", "q_axs6_layer",
-                 "q_e2m3_layer", "fq_axs6_grad", "exp_mxfp4_scores", "qcols_e2m3_weight", "exmy_e3m3_act"]
+                 "q_e2m3_layer", "fq_axs6_grad", "exp_mxfp4_scores", "expfree_mxfp4_scores", "qcols_e2m3_weight",
+                 "exmy_e3m3_act"]
 
 
 def profile_case(name, reps):
@@ -493,6 +497,10 @@ def profile_case(name, reps):
         sc = torch.randn(4096, 32768, device=dev, generator=gen) * 3
         c, s = mxq.exp_quantize(sc, "mxfp4")
         fn = lambda: mxq.exp_quantize(sc, "mxfp4", codes=c, scales=s)
+    elif name == "expfree_mxfp4_scores":
+        sc = torch.randn(4096, 32768, device=dev, generator=gen) * 3
+        c, s = mxq.exp_free_quantize(sc)
+        fn = lambda: mxq.exp_free_quantize(sc, codes=c, scales=s)
     else:
         raise SystemExit(f"unknown profile case {name}; one of {PROFILE_CASES}")
     for _ in range(reps):

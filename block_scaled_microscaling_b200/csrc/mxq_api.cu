@@ -304,6 +304,13 @@ mxq_status mxq_exp_quantize(mxq_format fmt, const float* scores, int64_t rows, i
     return from_cuda(mxq::launch_exp_quantize((int)fmt, scores, rows, cols, codes, scales, (cudaStream_t)stream));
 }
 
+mxq_status mxq_exp_free_quantize(const float* scores, int64_t rows, int64_t cols, void* codes, void* scales,
+                                 mxq_stream stream) {
+    MXQ_TRY(check_quantize_args(MXQ_MXFP4_E2M1, scores, MXQ_F32, rows, cols, codes, scales));
+    if (rows == 0) return MXQ_OK;
+    return from_cuda(mxq::launch_exp_free_quantize(scores, rows, cols, codes, scales, (cudaStream_t)stream));
+}
+
 mxq_status mxq_quantize_cols(mxq_format fmt, const void* src, mxq_dtype dtype, int64_t rows, int64_t cols,
                              void* codes, void* scales, mxq_stream stream) {
     if (!fmt_ok(fmt) || !dtype_ok(dtype)) return MXQ_ERR_INVALID_ARG;

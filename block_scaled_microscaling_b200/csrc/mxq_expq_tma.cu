@@ -74,9 +74,64 @@ __device__ __forceinline__ void named_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// ---- exp-free E2M1 rule ------------------------------------------------------------------
+//
+// "EFQ-Softmax: exp-free E2M1 probabilities", opening paragraph and the paragraph on the
+// per-block rule: each microscaling block takes an exponent-only scale from its local maximum,
+// normalizes the shifted scores with it and maps them to nonnegative E2M1 codes with one affine
+// rule; no exponential. The page gives no constants; the library's reading (the oracle states
+// the same rule independently):
+//   u = RN(RN(s - m) * L2E), u_max = max over the block, Es = clamp(floor(u_max) - 2, -127, 127),
+//   w = RN(2u - 2Es) (one fused multiply-add), code = clamp(rint(w) + 2, 0, 7), ties to even.
+// rint(w) + 2 for w clamped to [-2, 5] is the low byte of RN(w + 1.5 * 2^23 + 2); the codes of
+// eight keys leave as one word (key k in nibble k) through byte permutes.
+__device__ __forceinline__ void exp_free_block(const uint32_t (&w)[32], float m, long long blk, void* codes,
+                                               void* scales) {
+    unsigned long long u[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        u[i] = f2mul(f2sub(pk(__uint_as_float(w[2 * i]), __uint_as_float(w[2 * i + 1])), dup2(m)), dup2(kL2E));
+    float q[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        float a, b;
+        upk(u[i], a, b);
+        q[i] = max_nan(a, b);
+    }
+    float um = max3_nan(max3_nan(q[0], q[1], q[2]), max3_nan(q[3], q[4], q[5]), max3_nan(q[6], q[7], q[8]));
+    um = max3_nan(um, max3_nan(q[9], q[10], q[11]), max3_nan(q[12], q[13], max_nan(q[14], q[15])));
+    int fl;
+    asm("cvt.rmi.s32.f32 %0, %1;" : "=r"(fl) : "f"(um));  // floor; -inf saturates to INT_MIN
+    const int es = min(max(fl, -125), 129) - 2;
+    const bool nan_block = um != um;
+    const uint32_t byte = nan_block ? 0xFFu : (uint32_t)(es + 127);
+    const unsigned long long two = dup2(2.0f), off = dup2(-2.0f * (float)es), rnd = dup2(12582914.0f);
+    uint32_t c[32];  // low byte of each: the code
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        float a, b;
+        upk(f2fma(two, u[i], off), a, b);
+        a = fminf(fmaxf(a, -2.0f), 5.0f);
+        b = fminf(fmaxf(b, -2.0f), 5.0f);
+        upk(f2add(pk(a, b), rnd), a, b);
+        c[2 * i] = __float_as_uint(a);
+        c[2 * i + 1] = __float_as_uint(b);
+    }
+    uint32_t out[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t* k = c + 8 * j;
+        const uint32_t ev = __byte_perm(__byte_perm(k[0], k[2], 0x0040), __byte_perm(k[4], k[6], 0x0040), 0x5410);
+        const uint32_t od = __byte_perm(__byte_perm(k[1], k[3], 0x0040), __byte_perm(k[5], k[7], 0x0040), 0x5410);
+        out[j] = nan_block ? 0u : (ev | (od << 4));
+    }
+    st_stream_v4(reinterpret_cast<char*>(codes) + blk * 16, make_uint4(out[0], out[1], out[2], out[3]));
+    reinterpret_cast<uint8_t*>(scales)[blk] = (uint8_t)byte;
+}
+
 // ---- the kernel ---------------------------------------------------------------------------
 
-template <int F, int CW, int MW, int NS, int LEAD>
+template <int F, int CW, int MW, int NS, int LEAD, bool XF>
 __global__ void __launch_bounds__(32 * (CW + MW + 1), 1)
     k_exp_quantize_tma(const float* __restrict__ scores, void* codes, void* scales, long long rows, long long cols,
                        bool a32, unsigned int* err) {
@@ -182,7 +237,8 @@ __global__ void __launch_bounds__(32 * (CW + MW + 1), 1)
         for (long long b = tid; b < bpr; b += 32 * CW) {
             uint32_t w[32];
             load_block<float>(s, b, w, a32);
-            exp_quant_block<F>(w, m, row * bpr + b, codes, scales, a32);
+            if constexpr (XF) exp_free_block(w, m, row * bpr + b, codes, scales);
+            else exp_quant_block<F>(w, m, row * bpr + b, codes, scales, a32);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bfree[slot]));
@@ -206,10 +262,10 @@ bool exp_quantize_tma_supported(int fmt, const void* scores) {
     return (fmt == F_E2M1 || fmt == F_E4M3) && (reinterpret_cast<uintptr_t>(scores) & 15) == 0;
 }
 
-template <int F, int CW, int MW, int NS, int LEAD>
+template <int F, int CW, int MW, int NS, int LEAD, bool XF = false>
 static cudaError_t launch_xt(const float* scores, long long rows, long long cols, void* codes, void* scales,
                              cudaStream_t st) {
-    auto kern = k_exp_quantize_tma<F, CW, MW, NS, LEAD>;
+    auto kern = k_exp_quantize_tma<F, CW, MW, NS, LEAD, XF>;
     const int smem = NS * kXStageBytes, threads = 32 * (CW + MW + 1);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -232,6 +288,14 @@ cudaError_t launch_exp_quantize_tma(int fmt, const float* scores, long long rows
     if (fmt == F_E2M1) return launch_xt<F_E2M1, kXWarps, kXMaxWarps, kXStages, kXLead>(scores, rows, cols, codes, scales, st);
     if (fmt == F_E4M3) return launch_xt<F_E4M3, kXWarps, kXMaxWarps, kXStages, kXLead>(scores, rows, cols, codes, scales, st);
     return cudaErrorInvalidValue;
+}
+
+// The exp-free rule through the same pipeline (scores 16-byte aligned, cols % 32 == 0).
+cudaError_t launch_exp_free_quantize(const float* scores, long long rows, long long cols, void* codes, void* scales,
+                                     cudaStream_t st) {
+    if (rows == 0) return cudaSuccess;
+    if ((reinterpret_cast<uintptr_t>(scores) & 15) != 0 || cols <= 0 || cols % 32 != 0) return cudaErrorInvalidValue;
+    return launch_xt<F_E2M1, kXWarps, kXMaxWarps, kXStages, kXLead, true>(scores, rows, cols, codes, scales, st);
 }
 
 // Self-test of the bounded wait: one warp waits on an mbarrier that nothing

@@ -62,6 +62,8 @@ cudaError_t launch_exp_quantize(int fmt, const float* scores, long long rows, lo
 bool exp_quantize_supported(long long cols);
 // bulk-copy pipeline form of the softmax stage (E2M1 and E4M3, scores 16-byte aligned)
 bool exp_quantize_tma_supported(int fmt, const void* scores);
+cudaError_t launch_exp_free_quantize(const float* scores, long long rows, long long cols, void* codes, void* scales,
+                                     cudaStream_t st);
 cudaError_t launch_exp_quantize_tma(int fmt, const float* scores, long long rows, long long cols, void* codes,
                                     void* scales, cudaStream_t st);
 // the device error word (bit 0: a bounded wait in a kernel ran out): its device address for

@@ -3,7 +3,7 @@
 The functions named like the C entry points (mxq_quantize, ...) take raw
 integers (device pointers, sizes, a cudaStream_t handle) and return the
 mxq_status code. The torch-facing helpers below them (quantize, dequantize,
-fake_quantize, exp_quantize, quantize_grouped) only allocate outputs with
+fake_quantize, exp_quantize, exp_free_quantize, quantize_grouped) only allocate outputs with
 torch, read pointers/strides and the current stream, call the C entry point
 and raise MXQError on a non-zero status. Every step of the method runs in the
 CUDA kernels of libmxq; there is no CPU path: if libmxq.so is missing, every
@@ -22,7 +22,8 @@ STATUS = {0: "MXQ_OK", 1: "MXQ_ERR_INVALID_ARG", 2: "MXQ_ERR_SHAPE", 3: "MXQ_ERR
 MAX_GROUP = 64
 ELEM_BITS = {"axs6": 6, "mxfp6_e2m3": 6, "mxfp6_e3m2": 6, "mxfp8": 8, "mxfp4": 4}
 
-EXPORTS = ["mxq_quantize", "mxq_dequantize", "mxq_fake_quantize", "mxq_exp_quantize", "mxq_quantize_grouped",
+EXPORTS = ["mxq_quantize", "mxq_dequantize", "mxq_fake_quantize", "mxq_exp_quantize", "mxq_exp_free_quantize",
+           "mxq_quantize_grouped",
            "mxq_quantize_cols", "mxq_dequantize_cols", "mxq_quantize_exmy", "mxq_dequantize_exmy",
            "mxq_fake_quantize_exmy", "mxq_quantize_mma", "mxq_swizzle_scales", "mxq_mma_scales_bytes", "mxq_run_batch", "mxq_check_device", "mxq_selftest_timeout",
            "mxq_codes_bytes", "mxq_scales_bytes", "mxq_block_bits", "mxq_status_string",
@@ -63,6 +64,7 @@ def lib():
             ("mxq_dequantize", [i32, vp, vp, i64, i64, vp, i32, vp]),
             ("mxq_fake_quantize", [i32, vp, i32, i64, i64, vp, vp]),
             ("mxq_exp_quantize", [i32, vp, i64, i64, vp, vp, vp]),
+            ("mxq_exp_free_quantize", [vp, i64, i64, vp, vp, vp]),
             ("mxq_quantize_grouped", [i32, i32, ctypes.POINTER(_Tensor), i32, vp]),
             ("mxq_quantize_cols", [i32, vp, i32, i64, i64, vp, vp, vp]),
             ("mxq_dequantize_cols", [i32, vp, vp, i64, i64, vp, i32, vp]),
@@ -112,6 +114,10 @@ def mxq_fake_quantize(fmt, src, dtype, rows, cols, dst, stream):
 
 def mxq_exp_quantize(fmt, scores, rows, cols, codes, scales, stream):
     return lib().mxq_exp_quantize(fmt, scores, rows, cols, codes, scales, stream)
+
+
+def mxq_exp_free_quantize(scores, rows, cols, codes, scales, stream):
+    return lib().mxq_exp_free_quantize(scores, rows, cols, codes, scales, stream)
 
 
 def mxq_quantize_grouped(fmt, dtype, tensors, stream):
@@ -303,6 +309,22 @@ def exp_quantize(scores, fmt="mxfp4", codes=None, scales=None, stream=None):
         scales = empty_scales(fmt, rows, cols, scores.device)
     _check(mxq_exp_quantize(_fmt(fmt), scores.data_ptr(), rows, cols, codes.data_ptr(), scales.data_ptr(),
                             _stream(stream)), "mxq_exp_quantize")
+    return codes, scales
+
+
+def exp_free_quantize(scores, codes=None, scales=None, stream=None):
+    """fp32 scores [..., keys] -> MXFP4 codes + E8M0 scales by the exp-free rule (no exponential):
+    per 32 keys an exponent-only scale from the block's maximum, one affine map to E2M1 codes."""
+    torch = _torch()
+    if scores.dtype != torch.float32 or not scores.is_contiguous():
+        raise ValueError("scores must be contiguous float32")
+    rows, cols = _as2d(scores)
+    if codes is None:
+        codes = empty_codes("mxfp4", rows, cols, scores.device)
+    if scales is None:
+        scales = empty_scales("mxfp4", rows, cols, scores.device)
+    _check(mxq_exp_free_quantize(scores.data_ptr(), rows, cols, codes.data_ptr(), scales.data_ptr(), _stream(stream)),
+           "mxq_exp_free_quantize")
     return codes, scales
 
 

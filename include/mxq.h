@@ -143,6 +143,30 @@ MXQ_API mxq_status mxq_exp_quantize(mxq_format fmt, const float* scores, int64_t
                             void* codes, void* scales, mxq_stream stream);
 
 /*
+ * Exp-free E2M1 probabilities ("EFQ-Softmax: exp-free E2M1 probabilities",
+ * opening paragraph and the paragraph on the per-block rule): the shifted
+ * scores go straight to nonnegative MXFP4 codes; no exponential is evaluated.
+ * Per row r and block of 32 keys:
+ *   u_j   = RN(RN(scores[r, j] - m) * L2E)   (m = row maximum as above,
+ *                                             L2E = 1/ln 2 rounded to fp32:
+ *                                             u_j = log2 of exp(s_j - m))
+ *   Es    = clamp(floor(max_j u_j) - 2, -127, 127)   exponent-only block scale,
+ *           stored as the E8M0 byte Es + 127
+ *   code  = clamp(rint(RN(2 u_j - 2 Es)) + 2, 0, 7)  ties to even, sign bit 0
+ * The page fixes the rule's structure (scale from the block's local maximum,
+ * one affine rule per block) but not its constants; these are the straight
+ * line through E2M1's grid in the log domain (codes 2, 4, 6 = 1, 2, 4 exactly).
+ * A block holding a NaN stores 0xFF and codes 0. Output layout as
+ * mxq_quantize(MXQ_MXFP4_E2M1): codes [rows, cols/32 * 16] bytes (key 2i in
+ * the low nibble), scales [rows, cols/32] bytes; mxq_dequantize decodes them.
+ * scores 16-byte aligned, cols % 32 == 0; other rules and errors as
+ * mxq_exp_quantize. Runs on the bulk-copy pipeline of mxq_exp_quantize, whose
+ * waits are bounded (see mxq_check_device).
+ */
+MXQ_API mxq_status mxq_exp_free_quantize(const float* scores, int64_t rows, int64_t cols, void* codes, void* scales,
+                                         mxq_stream stream);
+
+/*
  * Grouped quantize: n independent tensors of one format and one value type
  * converted by a single launch (a decoder layer's seven weight matrices in the
  * online layer-by-layer conversion of "Sonar: Online MXFP6", Start a model).

@@ -30,7 +30,7 @@ def declared_symbols():
 
 def test_exports_every_declared_symbol(L):
     syms = declared_symbols()
-    assert len(syms) == 21
+    assert len(syms) == 22
     out = subprocess.run(["nm", "-D", "--defined-only", mxq.LIB_PATH], capture_output=True, text=True).stdout
     exported = set(re.findall(r"\bT\s+(mxq_\w+)", out))
     for s in syms:
