@@ -75,6 +75,7 @@ __device__ __forceinline__ float stage_max(uint32_t stage, int n16, int t) {
     return m;
 }
 
+// named barrier among the maximum warps (id 1)
 __device__ __forceinline__ void named_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -247,14 +248,19 @@ __global__ void __launch_bounds__(32 * (CW + MW + 1), 1)
     }
 
     if (warp >= CW) {  // maximum warps: pass A
+        // Every maximum warp executes one named barrier per row, also after one of its waits
+        // has given up (then it only keeps the barrier count: no warp can be left waiting).
         const int t = tid - 32 * CW, mw = warp - CW;
         long long k = 0;
+        bool alive = true;
         const float NEG_INF = __uint_as_float(0xFF800000u);
         for (long long i = 0; i < n; ++i) {
             float acc = NEG_INF;
             for (int j = 0; j < nc; ++j, ++k) {
+                if (!alive) continue;
                 const int s = (int)(k % NS);
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&full[s]), (uint32_t)(k / NS) & 1u, ab, err))) return;
+                alive = __all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&full[s]), (uint32_t)(k / NS) & 1u, ab, err));
+                if (!alive) continue;
                 acc = max_nan(acc, stage_max<NM>(ring0 + s * CH, chunk_bytes(j) / 16, t));
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
@@ -265,7 +271,7 @@ __global__ void __launch_bounds__(32 * (CW + MW + 1), 1)
             if (lane == 0) mpart[p][mw] = acc;
             if constexpr (MW > 1) named_sync(1, NM);
             else __syncwarp();
-            if (t == 0) {
+            if (t == 0 && !*ab) {
                 float m = mpart[p][0];
 #pragma unroll
                 for (int w = 1; w < MW; ++w) m = max_nan(m, mpart[p][w]);
@@ -297,24 +303,27 @@ __global__ void __launch_bounds__(32 * (CW + MW + 1), 1)
 
 // ---- the row-resident kernel (exp-free rule, rows of at most 128 KB) ----------------------
 //
-// The same three roles, but a row stays in the ring from its copy to its last code, so each
+// The same three roles, but a row stays in shared memory from its copy to its last code, so each
 // score crosses L2 -> SM once: the producer streams stage after stage of the CTA's rows (L2
 // evict_first: read once) into a ring of NS stages; the maximum warps fold each stage into the
-// row maximum as it lands and publish it (sixteen row slots); the consumers, in groups of
-// SB/128 threads taking the stages in turn, wait for the row's maximum, read their blocks from
-// shared memory (load_block_rot) and free each stage when done. A row of up to NS - 3 stages
-// leaves at least three stages streaming the next rows while the consumers work on it.
+// row maximum as it lands, meet at a named barrier per row, and their warp 0 publishes the row
+// maximum (sixteen row slots); the consumers, in groups of SB/128 threads taking the stages in
+// turn, wait for the row maximum, read their blocks from shared memory (load_block_rot) and free
+// each stage when done. A row of up to NS - 3 stages leaves at least three stages streaming the
+// next rows while the consumers work on it.
 // Measured on fp32 4096 x 32768 scores (fraction of the HBM copy peak): exp-free 0.93 here vs
-// 0.86 through L2; exp-then-quantize in this form 0.78 vs 0.81 through L2 (its exponentials
-// hold the resident row longer, so less of the ring streams), so it keeps the L2 kernel;
-// 16 KB stages 0.93 / 0.78, no better.
+// 0.86 through L2. Exp-then-quantize in this form 0.78 vs 0.81 through L2 (its exponentials hold
+// the resident row longer, so less of the ring streams), so it keeps the L2 kernel. 16 KB stages
+// were no better (0.93 / 0.78). Rows cut in halves across a two-CTA cluster, the halves' maxima
+// exchanged through distributed shared memory every row, were slower still (0.54 / 0.60: the
+// per-row coupling of the two CTAs stalls both).
 template <int CW, int MW, int NS, int SB>
 __global__ void __launch_bounds__(32 * (CW + MW + 1), 1)
     k_exp_free_res(const float* __restrict__ scores, void* codes, void* scales, long long rows, long long cols,
-                       unsigned int* err) {
+                   unsigned int* err) {
     constexpr int CH = SB, NM = 32 * MW, GT = SB / 128, NG = 32 * CW / GT;  // NG groups of GT threads
     static_assert(NG >= 1 && NG * GT == 32 * CW && GT % 32 == 0, "one consumer thread per block of a stage");
-    static_assert(NS <= 15, "sixteen row slots: the maximum warps run at most NS rows ahead of the consumers");
+    static_assert(NS <= 15, "sixteen row slots: no role runs more than NS rows ahead of the consumers");
     extern __shared__ __align__(128) uint8_t ring[];
     __shared__ __align__(8) unsigned long long full[NS], empty[NS], mready[16];
     __shared__ float mval[16], mpart[2][MW];
@@ -338,15 +347,14 @@ __global__ void __launch_bounds__(32 * (CW + MW + 1), 1)
     volatile int* ab = &abort_flag;
     const uint32_t ring0 = smem_u32(ring);
     auto chunk_bytes = [&](int j) { return (int)min((long long)CH, rowbytes - (long long)j * CH); };
-    const long long nk = n * nc;  // stages of this CTA
+    auto row_src = [&](long long i) { return reinterpret_cast<const char*>(scores) + (blockIdx.x + i * G) * rowbytes; };
 
-    if (warp == CW + MW) {  // producer
-        if (lane != 0) return;
+    auto producer = [&]() {
         const unsigned long long strm = l2_policy_stream();
         long long k = 0;
         bool ok = true;
         for (long long i = 0; i < n && ok; ++i) {
-            const char* src = reinterpret_cast<const char*>(scores) + (blockIdx.x + i * G) * rowbytes;
+            const char* src = row_src(i);
             for (int j = 0; j < nc; ++j, ++k) {
                 const int s = (int)(k % NS);
                 ok = mbar_wait(smem_u32(&empty[s]), ((uint32_t)(k / NS) & 1u) ^ 1u, ab, err);
@@ -356,7 +364,7 @@ __global__ void __launch_bounds__(32 * (CW + MW + 1), 1)
                 bulk_load(ring0 + s * CH, src + (long long)j * CH, bytes, smem_u32(&full[s]), strm);
             }
         }
-        if (!ok) {
+        if (!ok) {  // gave up: let the copies still in flight land before shared memory goes away
             for (long long q = k > NS ? k - NS : 0; q < k; ++q) {
                 const uint32_t bar = smem_u32(&full[q % NS]), par = (uint32_t)(q / NS) & 1u;
                 const unsigned long long t0 = global_ns();
@@ -364,60 +372,70 @@ __global__ void __launch_bounds__(32 * (CW + MW + 1), 1)
                 }
             }
         }
-        return;
-    }
+    };
 
-    if (warp >= CW) {  // maximum warps
+    auto max_warps = [&]() {
+        // one named barrier per row for every maximum warp, also after a wait has given up
+        // (then the warp only keeps the barrier count); thread 0 then combines and publishes
         const int t = tid - 32 * CW, mw = warp - CW;
         long long k = 0;
+        bool alive = true;
         const float NEG_INF = __uint_as_float(0xFF800000u);
         for (long long i = 0; i < n; ++i) {
             float acc = NEG_INF;
             for (int j = 0; j < nc; ++j, ++k) {
+                if (!alive) continue;
                 const int s = (int)(k % NS);
-                if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&full[s]), (uint32_t)(k / NS) & 1u, ab, err))) return;
-                acc = max_nan(acc, stage_max<NM, SB>(ring0 + s * CH, chunk_bytes(j) / 16, t));
+                alive = __all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&full[s]), (uint32_t)(k / NS) & 1u, ab, err));
+                if (alive) acc = max_nan(acc, stage_max<NM, SB>(ring0 + s * CH, chunk_bytes(j) / 16, t));
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) acc = max_nan(acc, __shfl_xor_sync(0xFFFFFFFFu, acc, o));
-            const int p = (int)(i & 1);
-            if (lane == 0) mpart[p][mw] = acc;
+            const int q = (int)(i & 15);
+            if (lane == 0) mpart[i & 1][mw] = acc;
             if constexpr (MW > 1) named_sync(1, NM);
             else __syncwarp();
-            if (t == 0) {
-                float m = mpart[p][0];
+            if (mw == 0 && alive && lane == 0 && !*ab) {
+                float m = mpart[i & 1][0];
 #pragma unroll
-                for (int w = 1; w < MW; ++w) m = max_nan(m, mpart[p][w]);
-                mval[i & 15] = m;
-                mbar_arrive(smem_u32(&mready[i & 15]));
+                for (int w = 1; w < MW; ++w) m = max_nan(m, mpart[i & 1][w]);
+                mval[q] = m;
+                mbar_arrive(smem_u32(&mready[q]));
             }
         }
-        (void)nk;
-        return;
-    }
+    };
 
-    // consumers: group g takes the stages k with k % NG == g; thread tl owns block tl of a stage
-    const int g = tid / GT, tl = tid - g * GT;
-    const uint32_t r = (uint32_t)(tl & 7);
-    for (long long i = 0; i < n; ++i) {
-        const int slot = (int)(i & 15);
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&mready[slot]), (uint32_t)(i >> 4) & 1u, ab, err))) return;
-        const float m = *reinterpret_cast<volatile float*>(&mval[slot]);
-        const long long row_blk = (blockIdx.x + i * G) * bpr;
-        for (int j = 0; j < nc; ++j) {
-            const long long k = i * nc + j;
-            if ((int)(k % NG) != g) continue;
-            const int s = (int)(k % NS);
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&full[s]), (uint32_t)(k / NS) & 1u, ab, err))) return;
-            if (tl < chunk_bytes(j) / 128) {
-                uint32_t w[32];
-                load_block_rot(ring0 + s * CH + 128u * (uint32_t)tl, r, w);
-                const long long b = row_blk + (long long)j * GT + tl;
-                exp_free_rot(w, r, m, b, codes, scales);
+    auto consumers = [&]() {  // group g takes the stages k with k % NG == g; thread tl owns block tl
+        const int g = tid / GT, tl = tid - g * GT;
+        const uint32_t r = (uint32_t)(tl & 7);
+        for (long long i = 0; i < n; ++i) {
+            const int q = (int)(i & 15);
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&mready[q]), (uint32_t)(i >> 4) & 1u, ab, err))) return;
+            const float m = *reinterpret_cast<volatile float*>(&mval[q]);
+            const long long blk0 = (blockIdx.x + i * G) * bpr;
+            for (int j = 0; j < nc; ++j) {
+                const long long k = i * nc + j;
+                if ((int)(k % NG) != g) continue;
+                const int s = (int)(k % NS);
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&full[s]), (uint32_t)(k / NS) & 1u, ab, err))) return;
+                if (tl < chunk_bytes(j) / 128) {
+                    uint32_t w[32];
+                    load_block_rot(ring0 + s * CH + 128u * (uint32_t)tl, r, w);
+                    const long long b = blk0 + (long long)j * GT + tl;
+                    exp_free_rot(w, r, m, b, codes, scales);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
         }
+    };
+
+    if (warp == CW + MW) {
+        if (lane == 0) producer();
+    } else if (warp >= CW) {
+        max_warps();
+    } else {
+        consumers();
     }
 }
 
@@ -439,7 +457,7 @@ bool exp_quantize_tma_supported(int fmt, const void* scores) {
 }
 
 // Row-resident shape (exp-free rule): 16 consumer warps, 2 maximum warps, a ring of kRStages
-// stages of kRStageBytes; rows of up to 128 KB (32768 fp32 keys) stay resident, longer rows
+// stages of kRStageBytes; rows of up to four stages (32768 fp32 keys) stay resident, longer rows
 // take the L2 kernel.
 constexpr int kRWarps = 16, kRMaxWarps = 2, kRStageBytes = 32768, kRStages = 7;
 
