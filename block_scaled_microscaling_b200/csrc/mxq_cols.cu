@@ -15,12 +15,16 @@
 // once its values are in registers) and leave as contiguous runs of the
 // column's row-blocks.
 #include <cstdint>
+#include <mutex>
+#include <cuda.h>  // CUtensorMap and its enums (types only: the encoder is fetched through the runtime)
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include "mxq_block.cuh"
 #include "mxq_device.cuh"
 #include "mxq_internal.h"
+#include "mxq_tma.cuh"
 
 namespace mxq {
 
@@ -175,6 +179,167 @@ __global__ void __launch_bounds__(kColThreads) k_quantize_cols(const void* __res
     }
 }
 
+// ---- quantize, persistent and fed by the tensor-copy engine ---------------------------------------
+//
+// The same tile and the same compute as k_quantize_cols, but each CTA walks its tiles (tile
+// blockIdx.x + n * gridDim.x) with two tile buffers: a 2-D tensor copy (cp.async.bulk.tensor,
+// 256 rows x 128 bytes, 128-byte swizzle) brings tile n + 2 while tile n + 1 waits and tile n is
+// encoded. The 128-byte swizzle stores 16-byte chunk c of tile row r at chunk c ^ (r mod 8) of a
+// 1024-byte-aligned buffer: exactly the layout gather_columns reads. No wave tail (a one-shot
+// grid of 256-row tiles covered 1.38 waves at 4096 x 4096) and no per-thread load instructions.
+// Waits are bounded (the library's device error word); on a timeout every thread leaves the
+// loop together and thread 0 lets the copies in flight land first.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<unsigned long long>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+constexpr int kTileBytes = kTileRows * kRowBytes;  // 32 KB
+
+template <int F, typename T> struct QColsSmem {
+    static constexpr int TC = ColTile<T>::TC, PB = payload<F>(), SB = Fmt<F>::FIXED ? 2 : 1;
+    static constexpr int CS = 8 * PB + 8;
+    static constexpr int bytes = 2 * kTileBytes + TC * CS + TC * 8 * SB + 1024;  // + alignment slack
+};
+
+template <int F, typename T>
+__global__ void __launch_bounds__(kColThreads) k_quantize_cols_tma(const __grid_constant__ CUtensorMap tmap,
+                                                                  void* __restrict__ codes, void* __restrict__ scales,
+                                                                  long long rows, long long cols, unsigned int* err) {
+    constexpr int TC = ColTile<T>::TC, CPL = ColTile<T>::CPL;
+    constexpr int PB = payload<F>();
+    constexpr int SB = Fmt<F>::FIXED ? 2 : 1;
+    constexpr int CS = 8 * PB + 8;
+    extern __shared__ uint8_t dsm[];
+    uint8_t* const tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm) + 1023) & ~uintptr_t(1023));
+    uint8_t* const out = tiles + 2 * kTileBytes;
+    uint8_t* const sc = out + TC * CS;
+    __shared__ __align__(8) unsigned long long full[2];
+    __shared__ int abort_flag;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const long long RB = rows / 32;
+    const long long nsx = (cols + TC - 1) / TC, ntiles = nsx * ((rows + kTileRows - 1) / kTileRows);
+    const long long G = gridDim.x;
+    if (t == 0) {
+        mbar_init(smem_u32(&full[0]), 1);
+        mbar_init(smem_u32(&full[1]), 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    volatile int* ab = &abort_flag;
+    long long issued = 0;  // thread 0: tiles whose copy has been issued
+    auto issue = [&](long long n) {
+        const long long tile = blockIdx.x + n * G;
+        if (tile >= ntiles) return;
+        const int b = (int)(n & 1);
+        mbar_expect_tx(smem_u32(&full[b]), kTileBytes);
+        tma_load_2d(smem_u32(tiles + b * kTileBytes), &tmap, (int)((tile % nsx) * TC), (int)((tile / nsx) * kTileRows),
+                    smem_u32(&full[b]));
+        issued = n + 1;
+    };
+    if (t == 0) {
+        issue(0);
+        issue(1);
+    }
+    long long n = 0;
+    for (;; ++n) {
+        const long long tile = blockIdx.x + n * G;
+        if (tile >= ntiles) break;
+        const int b = (int)(n & 1);
+        const bool ok = mbar_wait(smem_u32(&full[b]), (uint32_t)(n >> 1) & 1u, ab, err);
+        if (__syncthreads_or(!ok)) break;
+        const long long sx = tile % nsx, sy = tile / nsx;
+        const long long col0 = sx * TC, row0 = sy * kTileRows;
+        const int nrb = (int)min((long long)kTileRows, rows - row0) / 32;
+        const int ncols = (int)min((long long)TC, cols - col0);
+        uint32_t w[CPL][Blk<T>::NW];
+        if (warp < nrb) gather_columns<T>(tiles + b * kTileBytes, warp, lane, w);
+        __syncthreads();  // buffer b read by every warp, the previous tile's staged outputs stored
+        if (t == 0) issue(n + 2);
+        if (warp < nrb) {
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) {
+                const int j = lane * CPL + k;  // column within the strip
+                if (j < ncols) {
+                    const uint32_t byte = scale_byte<F>(block_amax<T>(w[k]));
+                    uint32_t o[8];
+                    encode_block<F, T>(w[k], byte, o);
+                    uint32_t* q = reinterpret_cast<uint32_t*>(out + j * CS + warp * PB);
+#pragma unroll
+                    for (int i = 0; i < PB / 4; ++i) q[i] = o[i];
+                    if constexpr (SB == 2) reinterpret_cast<uint16_t*>(sc)[j * 8 + warp] = (uint16_t)byte;
+                    else sc[j * 8 + warp] = (uint8_t)byte;
+                }
+            }
+        }
+        __syncthreads();
+        // column j's row-blocks of this tile are contiguous in the output: nrb * PB bytes
+        if (nrb == 8 && ncols == TC) {
+#pragma unroll
+            for (int i = t; i < TC * PB; i += kColThreads) {
+                const int j = i / PB, k = i % PB;
+                const long long g = ((col0 + j) * RB + sy * 8) * PB + 8 * k;
+                *reinterpret_cast<uint2*>(reinterpret_cast<char*>(codes) + g) = *reinterpret_cast<const uint2*>(out + j * CS + 8 * k);
+            }
+#pragma unroll
+            for (int i = t; i < TC * 8; i += kColThreads) {
+                const int j = i >> 3, k = i & 7;
+                const long long g = (col0 + j) * RB + sy * 8 + k;
+                if constexpr (SB == 2) reinterpret_cast<uint16_t*>(scales)[g] = reinterpret_cast<const uint16_t*>(sc)[j * 8 + k];
+                else reinterpret_cast<uint8_t*>(scales)[g] = sc[j * 8 + k];
+            }
+        } else {
+            const int seg8 = nrb * PB / 8;
+            for (int i = t; i < ncols * seg8; i += kColThreads) {
+                const int j = i / seg8, k = i % seg8;
+                const long long g = ((col0 + j) * RB + sy * 8) * PB + 8 * k;
+                *reinterpret_cast<uint2*>(reinterpret_cast<char*>(codes) + g) = *reinterpret_cast<const uint2*>(out + j * CS + 8 * k);
+            }
+            for (int i = t; i < ncols * nrb; i += kColThreads) {
+                const int j = i / nrb, k = i % nrb;
+                const long long g = (col0 + j) * RB + sy * 8 + k;
+                if constexpr (SB == 2) reinterpret_cast<uint16_t*>(scales)[g] = reinterpret_cast<const uint16_t*>(sc)[j * 8 + k];
+                else reinterpret_cast<uint8_t*>(scales)[g] = sc[j * 8 + k];
+            }
+        }
+    }
+    if (t == 0) {  // after a timeout: the copies issued and not consumed land before shared memory goes away
+        for (long long q = n; q < issued; ++q) {
+            const uint32_t bar = smem_u32(&full[q & 1]), par = (uint32_t)(q >> 1) & 1u;
+            const unsigned long long t0 = global_ns();
+            while (!mbar_test(bar, par) && global_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+    }
+}
+
+// Tensor map of a [rows, cols] matrix of 2- or 4-byte values: boxes of 256 rows x 128 bytes,
+// 128-byte swizzle. The encoder is the driver's, fetched once through the runtime.
+static bool encode_tile_map(CUtensorMap* m, const void* base, long long rows, long long cols, int esize) {
+    static PFN_cuTensorMapEncodeTiled fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(p);
+        else
+            cudaGetLastError();
+    });
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * (cuuint64_t)esize};
+    const cuuint32_t box[2] = {(cuuint32_t)(kRowBytes / esize), (cuuint32_t)kTileRows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base),
+              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ---- dequantize: 32-column tiles (64-byte bf16 rows) -------------------------------------------
 // The 128-byte-row tile above was slower for dequantize (bf16 16384x8192: 0.53 vs 0.62 of the
 // HBM peak), so dequantize keeps tiles of 256 rows x 32 columns, chunk c of row r at c ^ (r/2 mod 4)
@@ -296,6 +461,24 @@ template <int F, typename T>
 static cudaError_t launch_qc_t(const void* src, void* codes, void* scales, long long rows, long long cols,
                                cudaStream_t st) {
     constexpr int TC = ColTile<T>::TC;
+    CUtensorMap map;
+    if (encode_tile_map(&map, src, rows, cols, (int)sizeof(T))) {
+        auto kern = k_quantize_cols_tma<F, T>;
+        constexpr int smem = QColsSmem<F, T>::bytes;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        int dev = 0, sms = 148, per_sm = 1;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kColThreads, smem);
+        const long long ntiles = ((cols + TC - 1) / TC) * ((rows + kTileRows - 1) / kTileRows);
+        long long grid = (long long)sms * (per_sm > 0 ? per_sm : 1);
+        if (grid > ntiles) grid = ntiles;
+        unsigned int* err = nullptr;
+        if ((e = device_error_word(&err)) != cudaSuccess) return e;
+        kern<<<(unsigned)grid, kColThreads, smem, st>>>(map, codes, scales, rows, cols, err);
+        return cudaGetLastError();
+    }
     dim3 grid((unsigned)((cols + TC - 1) / TC), (unsigned)((rows + kTileRows - 1) / kTileRows));
     k_quantize_cols<F, T><<<grid, kColThreads, 0, st>>>(src, codes, scales, rows, cols);
     return cudaGetLastError();
