@@ -447,7 +447,7 @@ def workloads_breakdown(torch, mxq, hbm):
 
 PROFILE_CASES = ["batch_weight", "q_e2m3_weight", "q_e3m2_weight", "dq_e2m3_weight", "q_mxfp8_act", "dq_mxfp8_act", "q_axs6_layer",
                  "q_e2m3_layer", "fq_axs6_grad", "exp_mxfp4_scores", "expfree_mxfp4_scores", "qcols_e2m3_weight",
-                 "exmy_e3m3_act"]
+                 "dqcols_e2m3_weight", "exmy_e3m3_act", "dq_exmy_e3m3_act", "fq_exmy_e3m3_act", "qmma_mxfp8_act"]
 
 
 def profile_case(name, reps):
@@ -461,7 +461,7 @@ def profile_case(name, reps):
         w = torch.from_numpy(w_host.view(np.int16)).view(torch.bfloat16).cuda()
         sets = make_sets(torch, mxq, w, 8)
         fn = step_batch(mxq, sets, 0)
-    elif name in ("q_e2m3_weight", "q_e3m2_weight", "dq_e2m3_weight", "qcols_e2m3_weight"):
+    elif name in ("q_e2m3_weight", "q_e3m2_weight", "dq_e2m3_weight", "qcols_e2m3_weight", "dqcols_e2m3_weight"):
         w_host, _ = synthetic.weight_with_outliers(seed=1)
         x = torch.from_numpy(w_host.view(np.int16)).view(torch.bfloat16).cuda()
         f = "mxfp6_e3m2" if "e3m2" in name else "mxfp6_e2m3"
@@ -469,14 +469,27 @@ def profile_case(name, reps):
         y = torch.empty_like(x)
         if name.startswith("qcols"):
             fn = lambda: mxq.quantize_cols(x, f, codes=c, scales=s)
+        elif name.startswith("dqcols"):
+            cc, cs = mxq.quantize_cols(x, f)
+            fn = lambda: mxq.dequantize_cols(cc, cs, f, x.shape, out=y)
         elif name[0] == "q":
             fn = lambda: mxq.quantize(x, f, codes=c, scales=s)
         else:
             fn = lambda: mxq.dequantize(c, s, f, x.shape, out=y)
-    elif name == "exmy_e3m3_act":
+    elif name in ("exmy_e3m3_act", "dq_exmy_e3m3_act", "fq_exmy_e3m3_act"):
         x = (torch.randn(16384, 8192, device=dev, generator=gen) * 0.5).to(torch.bfloat16)
         c, s = mxq.quantize_exmy(x, 3, 3)
-        fn = lambda: mxq.quantize_exmy(x, 3, 3, codes=c, scales=s)
+        y = torch.empty_like(x)
+        if name == "exmy_e3m3_act":
+            fn = lambda: mxq.quantize_exmy(x, 3, 3, codes=c, scales=s)
+        elif name == "dq_exmy_e3m3_act":
+            fn = lambda: mxq.dequantize_exmy(c, s, 3, 3, x.shape, out=y)
+        else:
+            fn = lambda: mxq.fake_quantize_exmy(x, 3, 3, out=y)
+    elif name == "qmma_mxfp8_act":
+        x = (torch.randn(16384, 8192, device=dev, generator=gen) * 0.5).to(torch.bfloat16)
+        c, s = mxq.quantize_mma(x, "mxfp8")
+        fn = lambda: mxq.quantize_mma(x, "mxfp8", codes=c, scales=s)
     elif name in ("q_mxfp8_act", "dq_mxfp8_act"):
         x = (torch.randn(16384, 8192, device=dev, generator=gen) * 0.5).to(torch.bfloat16)
         c, s = mxq.quantize(x, "mxfp8")
