@@ -44,6 +44,7 @@ struct ExmyParams {
     uint32_t emin_b;  // 128 - b: biased fp32 exponent of the smallest normal 2^(1-b)
     uint32_t cadd;    // ((23 - M) << 23) | 0x400000: the rounding constant's bits less its exponent
     uint32_t kcode;   // (b - 128) << M (mod 2^32)
+    float maxval;     // value of the largest magnitude code
 };
 
 static ExmyParams exmy_params(int E, int M) {
@@ -67,6 +68,9 @@ static ExmyParams exmy_params(int E, int M) {
     p.emin_b = (uint32_t)(128 - b);
     p.cadd = ((uint32_t)(23 - M) << 23) | 0x400000u;
     p.kcode = (uint32_t)(b - 128) << M;
+    // largest magnitude: exponent field 2^E - 1, mantissa 2^M - 1 (E = 0: fixed point (2^M - 1) / 2^(M - 1))
+    p.maxval = E >= 1 ? ldexpf(1.0f + (float)((1 << M) - 1) / (float)(1 << M), (1 << E) - 1 - b)
+                      : (float)((1 << M) - 1) / (float)(1 << (M - 1));
     return p;
 }
 
@@ -81,6 +85,14 @@ __device__ __forceinline__ uint32_t exmy_mag(float y, const ExmyParams& p) {
     const uint32_t cb = eb * 0x800000u + p.cadd;
     const uint32_t q = __float_as_uint(y + __uint_as_float(cb)) - cb;
     return min((eb << p.M) + q + p.kcode, p.maxmag);
+}
+
+// The grid value nearest y >= 0 (already scaled), saturated: the same sum as exmy_mag, but the
+// rounded value is read back as RN(y + C) - C (exact: both lie in C's binade) instead of as a code.
+__device__ __forceinline__ float exmy_round_value(float y, const ExmyParams& p) {
+    const uint32_t eb = max(__float_as_uint(y) >> 23, p.emin_b);
+    const float c = __uint_as_float(eb * 0x800000u + p.cadd);
+    return fminf(__fsub_rn(__fadd_rn(y, c), c), p.maxval);
 }
 
 template <int W> __device__ __forceinline__ void pack_codes(const uint32_t* c, uint32_t* out) {
@@ -98,6 +110,13 @@ template <int W> __device__ __forceinline__ uint32_t code_of(const uint32_t* pw,
     uint32_t c = pw[wd] >> off;
     if (off + W > 32) c |= pw[wd + 1] << (32 - off);
     return c & ((1u << W) - 1u);
+}
+
+// sign bit (as an fp32 sign) of value k of a block held as words
+template <typename T> __device__ __forceinline__ uint32_t w2sign(const uint32_t* w, int k);
+template <> __device__ __forceinline__ uint32_t w2sign<float>(const uint32_t* w, int k) { return w[k] & 0x80000000u; }
+template <> __device__ __forceinline__ uint32_t w2sign<__nv_bfloat16>(const uint32_t* w, int k) {
+    return (k & 1) ? (w[k >> 1] & 0x80000000u) : ((w[k >> 1] << 16) & 0x80000000u);
 }
 
 // values of one block -> W payload words
@@ -217,9 +236,29 @@ __global__ void __launch_bounds__(kExThreads) k_fake_quantize_exmy(const void* s
         load_block<T>(src, b, w, a32);
         const uint32_t am = block_amax<T>(w);
         const uint32_t byte = am >= 0x7F800000u ? 0xFFu : (uint32_t)max((int)(am >> 23) - p.emax, 0);
-        uint32_t pw[W], o[Blk<T>::NW];
-        exmy_encode<W, T>(w, byte, p, pw);
-        exmy_decode<W, T>(pw, byte, p, o);
+        // no codes: each value goes straight to its grid value, times the block scale, sign copied
+        // (bit-identical to decoding the encoded block)
+        const unsigned long long inv = dup2(inv_scale(byte == 0xFFu ? 0u : byte)), fwd = dup2(fwd_scale(byte == 0xFFu ? 0u : byte));
+        uint32_t o[Blk<T>::NW];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float a, c;
+            upk(f2mul(pair<T>(w, i), inv), a, c);
+            const float ra = exmy_round_value(fabsf(a), p), rc = exmy_round_value(fabsf(c), p);
+            upk(f2mul(pk(ra, rc), fwd), a, c);
+            a = __uint_as_float(__float_as_uint(a) | (w2sign<T>(w, 2 * i)));
+            c = __uint_as_float(__float_as_uint(c) | (w2sign<T>(w, 2 * i + 1)));
+            if constexpr (sizeof(T) == 4) {
+                o[2 * i] = __float_as_uint(a);
+                o[2 * i + 1] = __float_as_uint(c);
+            } else {
+                o[i] = bf16x2(a, c);
+            }
+        }
+        if (byte == 0xFFu) {
+#pragma unroll
+            for (int i = 0; i < Blk<T>::NW; ++i) o[i] = sizeof(T) == 4 ? 0x7FC00000u : 0x7FC07FC0u;
+        }
         store_block<T>(dst, b, o, a32);
     }
 }
