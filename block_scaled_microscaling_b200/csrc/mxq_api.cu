@@ -408,7 +408,7 @@ const char* mxq_status_string(mxq_status s) {
         case MXQ_ERR_INVALID_ARG: return "invalid argument (format, type, or a null/host/other-device/overlapping pointer)";
         case MXQ_ERR_SHAPE: return "invalid shape (rows < 0, cols <= 0, cols not a multiple of 32, or too large)";
         case MXQ_ERR_ALIGN: return "misaligned pointer (values and codes need 16 bytes, AXS-6 headers 2)";
-        case MXQ_ERR_UNSUPPORTED: return "valid request that this build does not support";
+        case MXQ_ERR_UNSUPPORTED: return "valid request that the library does not support";
         case MXQ_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
         case MXQ_ERR_TIMEOUT: return "a bounded device-side wait gave up";
     }

@@ -83,7 +83,7 @@ typedef enum {
     MXQ_ERR_INVALID_ARG = 1, /* bad enum, null / host / other-device pointer          */
     MXQ_ERR_SHAPE = 2,       /* rows < 0, cols <= 0, cols % 32 != 0, size overflow    */
     MXQ_ERR_ALIGN = 3,       /* a pointer misses its alignment (see each call)        */
-    MXQ_ERR_UNSUPPORTED = 4, /* valid request this build does not implement           */
+    MXQ_ERR_UNSUPPORTED = 4, /* valid request the library does not implement         */
     MXQ_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed                  */
     MXQ_ERR_TIMEOUT = 6      /* a bounded device-side wait gave up (reserved)         */
 } mxq_status;

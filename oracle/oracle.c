@@ -428,7 +428,7 @@ int orc_fake_quantize_exmy(int E, int M, const void* src, int dtype, int64_t row
  * higher precision (fp32 here), materialized, then quantized per 32-key block
  * to MXFP4 (E2M1 codes, exponent-only block scale).
  *
- * The exponential is this build's own deterministic fp32 function, defined
+ * The exponential is the method's own deterministic fp32 function, defined
  * so that any two faithful implementations agree bit for bit:
  *   t  = RN(d * L2E)                  L2E    = 1/ln 2 rounded to fp32
  *   n  = t rounded to an integer, ties to even
