@@ -45,6 +45,12 @@ struct ExmyParams {
     uint32_t cadd;    // ((23 - M) << 23) | 0x400000: the rounding constant's bits less its exponent
     uint32_t kcode;   // (b - 128) << M (mod 2^32)
     float maxval;     // value of the largest magnitude code
+    // the two-values-per-word path (bf16 values, M <= 5), every constant in both 16-bit lanes:
+    uint32_t emin2;   // (128 - b) << 7: bf16 exponent field of 2^(1-b)
+    uint32_t cadd2;   // ((7 - M) << 7) | 0x40: added to an exponent field, the bf16 bits of 1.5 * 2^(e + 7 - M)
+    uint32_t kneg2;   // -(((128 - b) << M) in both lanes): the code's exponent offset
+    uint32_t max2;    // maxmag
+    uint32_t sh7;     // 7 - M
 };
 
 static ExmyParams exmy_params(int E, int M) {
@@ -71,6 +77,12 @@ static ExmyParams exmy_params(int E, int M) {
     // largest magnitude: exponent field 2^E - 1, mantissa 2^M - 1 (E = 0: fixed point (2^M - 1) / 2^(M - 1))
     p.maxval = E >= 1 ? ldexpf(1.0f + (float)((1 << M) - 1) / (float)(1 << M), (1 << E) - 1 - b)
                       : (float)((1 << M) - 1) / (float)(1 << (M - 1));
+    auto both = [](uint32_t v) { return v | (v << 16); };
+    p.emin2 = both((uint32_t)(128 - b) << 7);
+    p.cadd2 = M <= 7 ? both(((uint32_t)(7 - M) << 7) | 0x40u) : 0u;
+    p.kneg2 = 0u - both((uint32_t)(128 - b) << M);
+    p.max2 = both(p.maxmag);
+    p.sh7 = M <= 7 ? (uint32_t)(7 - M) : 0u;
     return p;
 }
 
@@ -138,6 +150,68 @@ __device__ __forceinline__ void exmy_encode(const uint32_t* w, uint32_t byte, co
     }
 }
 
+// ---- bf16 values, M <= 5: two values per 32-bit word --------------------------------------
+//
+// The same rounding as exmy_mag, on the two bf16 values of a word at once: y = x * 2^-Es with
+// mul.rn.bf16x2 (exact: a power of two times an 8-bit significand; a result below bf16's normal
+// range is far below half the format's smallest step, so it still gives code 0), the binade
+// constant C = 1.5 * 2^(e + 7 - M) built in each 16-bit lane from y's exponent field (clamped
+// from below with max.u16x2), RN(y + C) with add.rn.bf16x2 (bf16's 8-bit significand puts
+// C's ulp at the grid step 2^(e - M), and y + C stays in C's binade while M <= 5), then the step
+// count q = bits(sum) - bits(C) and code = (e << M) + q - ((128 - b) << M) in 32-bit integer
+// adds: every lane's partial results lie in [0, 2^16), so no carry or borrow crosses lanes.
+// Saturation with min.u16x2, signs moved from bits 15/31 to bits W-1 / W+15.
+__device__ __forceinline__ uint32_t bf2mul(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ __forceinline__ uint32_t bf2add(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ __forceinline__ uint32_t umax2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ __forceinline__ uint32_t umin2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// 16 fields of 2W bits (codes of values 2i, 2i+1) -> W payload words, LSB-first
+template <int W> __device__ __forceinline__ void pack_pairs(const uint32_t* f, uint32_t* out) {
+#pragma unroll
+    for (int i = 0; i < W; ++i) out[i] = 0;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const int bit = 2 * W * k, wd = bit >> 5, off = bit & 31;
+        out[wd] |= f[k] << off;
+        if (off + 2 * W > 32) out[wd + 1] |= f[k] >> (32 - off);
+    }
+}
+
+template <int W>
+__device__ __forceinline__ void exmy_encode_bf16x2(const uint32_t* w, uint32_t byte, const ExmyParams& p, uint32_t* out) {
+    const uint32_t s = ((254u - byte) << 7) * 0x10001u;  // 2^(127 - byte) in both lanes; byte <= 253
+    constexpr uint32_t kSign = (1u << (W - 1)) | (1u << (W + 15));
+    uint32_t f[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint32_t y = bf2mul(w[i], s) & 0x7FFF7FFFu;
+        const uint32_t e = umax2(y & 0x7F807F80u, p.emin2);
+        const uint32_t c = e + p.cadd2;
+        const uint32_t q = bf2add(y, c) - c;
+        uint32_t code = umin2((e >> p.sh7) + q + p.kneg2, p.max2);
+        code |= (w[i] >> (16 - W)) & kSign;
+        f[i] = code - (code >> 16) * (65536u - (1u << W));  // c0 | c1 << W
+    }
+    pack_pairs<W>(f, out);
+}
+
 // W payload words -> 32 output values (bf16 pairs or fp32 words)
 template <int W, typename T>
 __device__ __forceinline__ void exmy_decode(const uint32_t* pw, uint32_t byte, const ExmyParams& p, uint32_t* o) {
@@ -180,7 +254,9 @@ __device__ __forceinline__ void warp_load_words(const void* codes, long long fir
     __syncwarp();
 }
 
-template <int W, typename T>
+// SW: the two-values-per-word rounding (bf16 values, M <= 5); a block whose scale byte is 254
+// (2^-127, not a normal bf16) or 0xFF takes the fp32 path
+template <int W, typename T, bool SW = false>
 __global__ void __launch_bounds__(kExThreads) k_quantize_exmy(const void* __restrict__ src, void* __restrict__ codes,
                                                               uint8_t* __restrict__ scales, long long nblocks,
                                                               ExmyParams p, bool a32) {
@@ -191,7 +267,12 @@ __global__ void __launch_bounds__(kExThreads) k_quantize_exmy(const void* __rest
         const uint32_t am = block_amax<T>(w);
         const uint32_t byte = am >= 0x7F800000u ? 0xFFu : (uint32_t)max((int)(am >> 23) - p.emax, 0);
         uint32_t out[W];
-        exmy_encode<W, T>(w, byte, p, out);
+        if constexpr (SW) {
+            if (byte <= 253u) exmy_encode_bf16x2<W>(w, byte, p, out);
+            else exmy_encode<W, T>(w, byte, p, out);
+        } else {
+            exmy_encode<W, T>(w, byte, p, out);
+        }
         char* q = reinterpret_cast<char*>(codes) + b * 4 * W;
         if constexpr (W == 4 || W == 8) {  // 16 or 32 bytes per lane: whole 16-byte stores
 #pragma unroll
@@ -264,10 +345,11 @@ __global__ void __launch_bounds__(kExThreads) k_fake_quantize_exmy(const void* s
 }
 
 // Grid: one CTA per 256 blocks (one pass: the hardware starts a CTA wherever one finishes) for
-// dequantize and fake-quantize, SMs x resident CTAs walking grid-stride for quantize. Measured
-// on bf16 16384x8192 over five splits (fraction of the copy peak): dequantize 0.85-0.94 ->
-// 0.90-0.93, fake-quantize 0.67-0.70 -> 0.70-0.72 with one pass; quantize, bound by its integer
-// rounding, 0.62-0.74 persistent vs 0.62-0.68 in one pass.
+// dequantize, fake-quantize and the two-lane bf16 quantize; SMs x resident CTAs walking
+// grid-stride for the fp32 quantize. Measured on bf16 16384x8192 over five splits (fraction of
+// the copy peak): dequantize 0.85-0.94 -> 0.90-0.93 with one pass; the two-lane quantize
+// 0.89-0.97 in one pass vs 0.64-0.87 persistent; the quantize on fp32 arithmetic, bound by its
+// integer rounding, 0.62-0.74 persistent vs 0.62-0.68 in one pass.
 static int ex_grid(const void* fn, long long nb, bool one_pass) {
     long long want = (nb + kExThreads - 1) / kExThreads;
     if (want < 1) want = 1;
@@ -288,8 +370,11 @@ static cudaError_t ex_launch(int op, const void* in, void* out, const void* aux_
                              const ExmyParams& p, cudaStream_t st) {
     if (op == 0) {
         auto k = k_quantize_exmy<W, T>;
-        k<<<ex_grid((const void*)k, nb, false), kExThreads, 0, st>>>(in, out, reinterpret_cast<uint8_t*>(aux_out), nb, p,
-                                                            al32(in, in));
+        bool two_lane = false;
+        if constexpr (sizeof(T) == 2) two_lane = p.M <= 5;
+        if (two_lane) k = k_quantize_exmy<W, T, true>;
+        k<<<ex_grid((const void*)k, nb, two_lane), kExThreads, 0, st>>>(in, out, reinterpret_cast<uint8_t*>(aux_out), nb,
+                                                                      p, al32(in, in));
     } else if (op == 1) {
         auto k = k_dequantize_exmy<W, T>;
         k<<<ex_grid((const void*)k, nb, true), kExThreads, 0, st>>>(in, reinterpret_cast<const uint8_t*>(aux_in), out, nb, p,
