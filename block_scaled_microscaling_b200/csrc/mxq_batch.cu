@@ -72,6 +72,7 @@ __device__ __forceinline__ void tile_fake_quantize(const BatchOp& op, long long 
 
 template <typename T>
 __global__ void __launch_bounds__(kBThreads) k_batch(const __grid_constant__ BatchTable tab) {
+    pdl_wait_then_release();
     __shared__ __align__(16) uint8_t stage[kBWarps][32 * 24];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const long long nwarps = (long long)gridDim.x * kBWarps;
@@ -113,11 +114,9 @@ cudaError_t launch_batch(int dtype, BatchTable& tab, cudaStream_t st) {
     long long grid = resident_ctas(fn, dev);
     const long long want = (tiles + kBWarps - 1) / kBWarps;
     if (want < grid) grid = want;
-    if (dtype == 1)
-        k_batch<__nv_bfloat16><<<(unsigned)grid, kBThreads, 0, st>>>(tab);
-    else
-        k_batch<float><<<(unsigned)grid, kBThreads, 0, st>>>(tab);
-    return cudaGetLastError();
+    const cudaError_t e = dtype == 1 ? launch_pdl(k_batch<__nv_bfloat16>, (unsigned)grid, kBThreads, st, tab)
+                                     : launch_pdl(k_batch<float>, (unsigned)grid, kBThreads, st, tab);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace mxq

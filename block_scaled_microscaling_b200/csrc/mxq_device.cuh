@@ -85,6 +85,15 @@ __device__ __forceinline__ void st32(void* p, const uint32_t* r, bool a32) {
 }
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch: wait for the grids this one depends on (before any global
+// memory access), then let the next launch in the stream be scheduled
+
+__device__ __forceinline__ void pdl_wait_then_release() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // packed fp32 pair arithmetic (one instruction for two IEEE round-to-nearest ops)
 
 __device__ __forceinline__ unsigned long long pk(float a, float b) {

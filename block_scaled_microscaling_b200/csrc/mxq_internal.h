@@ -66,6 +66,26 @@ cudaError_t launch_exp_free_quantize(const float* scores, long long rows, long l
                                      cudaStream_t st);
 cudaError_t launch_exp_quantize_tma(int fmt, const float* scores, long long rows, long long cols, void* codes,
                                     void* scales, cudaStream_t st);
+// Launch with programmatic stream serialization: the kernel may be scheduled while the previous
+// kernel of the stream drains; it waits for it (griddepcontrol.wait) before touching memory and
+// then lets the next launch be scheduled. Measured on back-to-back launches (fraction of the
+// copy peak): batch step 0.91 -> 0.92, single-tensor quantize at 47 MB +2% (MXFP8 +6%), at
+// 268 MB +0.5-1%. Used for the batch kernel, quantize and the one-pass dequantize.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(block, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute a[1];
+    a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = a;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // the device error word (bit 0: a bounded wait in a kernel ran out): its device address for
 // kernel arguments, and its value (clear resets it)
 cudaError_t device_error_word(unsigned int** p);
