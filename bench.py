@@ -607,7 +607,7 @@ def main():
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "u32", "data": "synthetic",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": WORKLOAD, "elements": n, "bytes_per_step": step_bytes,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "8 rotating buffer sets (~1 GB): each launch reads data last touched >= 4 steps earlier",
