@@ -136,8 +136,8 @@ MXQ_API mxq_status mxq_fake_quantize(mxq_format fmt, const void* src, mxq_dtype 
  *   then p is block-quantized exactly like mxq_quantize with dtype MXQ_F32.
  * p is never written to memory. Supported formats: all five (MXFP4 E2M1 is
  * the one the stage feeds). scores 16-byte aligned; any cols % 32 == 0.
- * MXFP4 and MXFP8 run as a bulk-copy (TMA) pipeline whose waits are bounded;
- * see mxq_check_device.
+ * Runs as a bulk-copy (TMA) pipeline whose waits are bounded; see
+ * mxq_check_device.
  */
 MXQ_API mxq_status mxq_exp_quantize(mxq_format fmt, const float* scores, int64_t rows, int64_t cols,
                             void* codes, void* scales, mxq_stream stream);
