@@ -130,7 +130,7 @@ mxq_status mxq_quantize(mxq_format fmt, const void* src, mxq_dtype dtype, int64_
     MXQ_TRY(check_quantize_args(fmt, src, dtype, rows, cols, codes, scales));
     if (rows == 0) return MXQ_OK;
     mxq::SegTable<1> tab{};
-    tab.seg[0] = {src, codes, scales, rows * (cols / 32), 0};
+    tab.seg[0] = {src, codes, scales, rows * (cols / 32), 0, 0};
     tab.n = 1;
     return from_cuda(mxq::launch_quantize<1>((int)fmt, (int)dtype, tab, (cudaStream_t)stream));
 }
@@ -185,7 +185,7 @@ mxq_status mxq_quantize_grouped(mxq_format fmt, mxq_dtype dtype, const mxq_tenso
         const mxq_tensor& t = tensors[i];
         MXQ_TRY(check_quantize_args(fmt, t.src, dtype, t.rows, t.cols, t.codes, t.scales));
         if (t.rows == 0) continue;
-        tab.seg[m++] = {t.src, t.codes, t.scales, t.rows * (t.cols / 32), 0};
+        tab.seg[m++] = {t.src, t.codes, t.scales, t.rows * (t.cols / 32), 0, 0};
     }
     if (m == 0) return MXQ_OK;
     tab.n = m;
