@@ -3,6 +3,7 @@ import numpy as np
 import pytest
 
 import oracle
+import synthetic
 
 torch = pytest.importorskip("torch")
 from block_scaled_microscaling_b200 import mxq  # noqa: E402
@@ -56,3 +57,26 @@ def test_unsupported_split():
     st = torch.cuda.current_stream().cuda_stream
     assert mxq.mxq_quantize_exmy(6, 2, x.data_ptr(), 0, 1, 32, c.data_ptr(), s.data_ptr(), st) == 4
     assert mxq.mxq_quantize_exmy(1, 8, x.data_ptr(), 0, 1, 32, c.data_ptr(), s.data_ptr(), st) == 4
+
+
+@pytest.mark.parametrize("E,M", [s for s in SPLITS if s[1] <= 5])
+def test_bf16_two_values_per_word_path_at_scale(E, M):
+    """bf16 values with M <= 5 round two values per 32-bit word (bf16x2 arithmetic, 16-bit
+    lanes): a 2048x8192 tensor with per-block exponents over +-60 binades, zero, -0 and
+    subnormal blocks, quantized whole; 48 sampled rows equal the oracle bit for bit."""
+    rng = np.random.default_rng(1000 + 10 * E + M)
+    rows, cols = 2048, 8192
+    nb = rows * cols // 32
+    x = rng.standard_normal((nb, 32)) * 2.0 ** rng.integers(-60, 61, nb)[:, None]
+    kind = rng.integers(0, 32, nb)
+    x[kind == 0] = 0.0
+    x[kind == 1] = -0.0
+    x[kind == 2] *= 2.0 ** -70  # bf16 subnormals
+    ties = rng.integers(-64, 65, (nb, 32)) * 2.0 ** rng.integers(-10, 10, nb)[:, None]
+    x = np.where((kind == 3)[:, None], ties, x)
+    h = synthetic.f32_to_bf16_bits(x.astype(np.float32).reshape(rows, cols))
+    codes, scales = mxq.quantize_exmy(dev(h), E, M)
+    sel = np.sort(rng.choice(rows, 48, replace=False))
+    oc, os_ = oracle.quantize_exmy(np.ascontiguousarray(h[sel]), E, M)
+    assert np.array_equal(host(scales)[sel], os_)
+    assert np.array_equal(host(codes)[sel], oc)
