@@ -11,7 +11,9 @@ ml_dtypes, integer steps in uint32 words, so a carry between the lanes would sho
 and compared, lane by lane, with the oracle's nearest-code rounding of the exact |x| / 2^(byte -
 127), for every finite bf16 magnitude, every split with M <= 5 and scale bytes across the range,
 restricted to what a block can hold (|x| / 2^(byte - 127) < 2^(emax + 1): the block maximum
-fixes the byte). A CPU proof of the method's exactness; the GPU tests check the kernels."""
+fixes the byte). Also the fused eXmY fake-quantize's grid value, r = RN(RN(y + C) - C) in fp32
+with C = 1.5 * 2^(e + 23 - M), clamped: equal to the decoded nearest code for every split. CPU
+checks of the recipes' exactness; the GPU tests check the kernels that implement them."""
 import ml_dtypes
 import numpy as np
 import pytest
@@ -21,7 +23,6 @@ import oracle
 SPLITS = [(E, M) for W in range(3, 10) for E in range(0, 6) for M in [W - 1 - E]
           if oracle.exmy_valid(E, M) and M <= 5]
 BYTES = [0, 1, 2, 3, 10, 60, 100, 118, 124, 125, 126, 127, 128, 129, 130, 134, 140, 170, 200, 250, 253]
-BOTH = np.uint32(0x10001)
 
 
 def bf16_bits_to_f64(h):
@@ -107,3 +108,33 @@ def test_the_recipe_needs_m_at_most_5():
     got_lo, _ = lanes(two_lane_codes(join(mags, np.zeros_like(mags)), byte, E, M))
     want = oracle.exmy_round_mags(E, M, bf16_bits_to_f64(mags))
     assert not np.array_equal(got_lo, want)
+
+
+ALL_SPLITS = [(E, M) for W in range(3, 10) for E in range(0, 6) for M in [W - 1 - E] if oracle.exmy_valid(E, M)]
+
+
+def round_value_recipe(y, E, M):
+    """The fused fake-quantize's grid value, emulated in fp32 (numpy float32 arithmetic rounds to
+    nearest even): C = 1.5 * 2^(e + 23 - M) with e = max(exponent of y, 1 - b), r = (y + C) - C,
+    clamped to the largest value."""
+    b = (1 << (E - 1)) - 1 if E >= 1 else 0
+    emin_b = np.uint32(128 - b)
+    cadd = np.uint32(((23 - M) << 23) | 0x400000)
+    eb = np.maximum(y.view(np.uint32) >> np.uint32(23), emin_b)
+    c = (eb * np.uint32(0x800000) + cadd).view(np.float32)
+    r = (y + c) - c
+    return np.minimum(r, np.float32(oracle.exmy_maxval(E, M)))
+
+
+@pytest.mark.parametrize("E,M", ALL_SPLITS)
+def test_fused_fake_quantize_value_equals_decoded_nearest_code(E, M):
+    emax = oracle.exmy_emax(E, M)
+    table = oracle.exmy_decode_table(E, M)
+    x = bf16_bits_to_f64(np.arange(0x7F80, dtype=np.uint32))
+    for byte in BYTES:
+        y64 = x * 2.0 ** (127 - byte)
+        y64 = y64[y64 < 2.0 ** (emax + 1)]
+        y = y64.astype(np.float32)
+        got = round_value_recipe(y, E, M).astype(np.float64)
+        want = table[oracle.exmy_round_mags(E, M, y64)]
+        assert np.array_equal(got, want), (E, M, byte)
