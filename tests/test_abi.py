@@ -130,3 +130,36 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(mxq, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         mxq.lib()
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include "mxq.h"
+
+/* a plain C caller of the ABI, linked against libmxq.so: the host-only queries */
+int main(void) {
+    printf("%zu %zu %zu %d %d %s\n", mxq_codes_bytes(MXQ_MXFP6_E2M3, 4096, 4096),
+           mxq_scales_bytes(MXQ_AXS6, 4096, 4096), mxq_codes_bytes(MXQ_MXFP4_E2M1, 3, 96),
+           mxq_block_bits(MXQ_AXS6), mxq_block_bits(MXQ_MXFP8_E4M3), mxq_status_string(MXQ_ERR_SHAPE));
+    return 0;
+}
+"""
+
+
+def test_plain_c_caller(L, tmp_path):
+    """The boundary is a C ABI: a C99 program built against include/mxq.h alone (no CUDA headers)
+    links with libmxq.so and calls it. Host-only queries; no kernel runs."""
+    src = tmp_path / "caller.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(mxq.LIB_PATH)
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                        os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir, "-lmxq",
+                        "-Wl,-rpath," + libdir], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out.stderr
+    a, b, c, d, e, msg = out.stdout.split(" ", 5)
+    assert int(a) == 4096 * 4096 // 32 * 24 and int(b) == 4096 * 4096 // 32 * 2 and int(c) == 3 * 3 * 16
+    assert int(d) == 202 and int(e) == 264
+    assert msg.strip() == mxq.mxq_status_string(2)
