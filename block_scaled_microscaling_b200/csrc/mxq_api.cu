@@ -225,7 +225,10 @@ mxq_status mxq_run_batch(mxq_dtype dtype, const mxq_op* ops, int n, mxq_stream s
         const mxq_op& o = ops[i];
         const mxq_format f = (mxq_format)o.fmt;
         if (!fmt_ok(f)) return MXQ_ERR_INVALID_ARG;
-        const size_t nv = (size_t)o.rows * (size_t)(o.cols > 0 ? o.cols : 0) * dtype_bytes(dtype);
+        // shapes are checked before any size is formed from them
+        const mxq_status shape = check_shape(o.rows, o.cols);
+        if (shape != MXQ_OK) return o.kind < MXQ_OP_QUANTIZE || o.kind > MXQ_OP_FAKE_QUANTIZE ? MXQ_ERR_INVALID_ARG : shape;
+        const size_t nv = (size_t)o.rows * (size_t)o.cols * dtype_bytes(dtype);
         mxq::BatchOp b{};
         b.kind = o.kind;
         b.fmt = o.fmt;

@@ -85,7 +85,7 @@ typedef enum {
     MXQ_ERR_ALIGN = 3,       /* a pointer misses its alignment (see each call)        */
     MXQ_ERR_UNSUPPORTED = 4, /* valid request the library does not implement         */
     MXQ_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed                  */
-    MXQ_ERR_TIMEOUT = 6      /* a bounded device-side wait gave up (reserved)         */
+    MXQ_ERR_TIMEOUT = 6      /* a bounded device-side wait gave up (mxq_check_device) */
 } mxq_status;
 
 /* A cudaStream_t, passed as an opaque pointer so this header needs no CUDA headers. */
@@ -292,10 +292,12 @@ MXQ_API mxq_status mxq_swizzle_scales(const void* scales, int64_t rows, int64_t 
                                       mxq_stream stream);
 
 /*
- * Device-side status. The bulk-copy pipeline behind mxq_exp_quantize (MXFP4 /
- * MXFP8) waits on its own asynchronous copies; every such wait is bounded (one
- * second). A wait that runs out makes the kernel stop early, leaving its
- * outputs incomplete, and sets a device error word. mxq_check_device
+ * Device-side status. The kernels that move data with the bulk-copy (TMA)
+ * engine wait on their own asynchronous copies: mxq_exp_quantize and
+ * mxq_exp_free_quantize (every format and size), mxq_quantize_cols, and
+ * mxq_fake_quantize on tensors of 2^19 blocks or more. Every such wait is
+ * bounded (one second). A wait that runs out makes the kernel stop early,
+ * leaving its outputs incomplete, and sets a device error word. mxq_check_device
  * synchronizes the current device and returns MXQ_ERR_TIMEOUT if that
  * happened since the last call (clearing the word), MXQ_ERR_CUDA if the device
  * reported an error, MXQ_OK otherwise. It is host-blocking; call it where a

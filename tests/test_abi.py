@@ -106,6 +106,36 @@ def test_statuses_before_any_cuda_call(L):
     assert b(1, [(1, 1, 0, 0, 0, 0, 2, 48)], None) == 2                 # cols % 32
     assert b(1, [(0, 1, 0, 0, 0, 0, 0, 64), (2, 0, 0, 0, 0, 0, 0, 32)], None) == 0  # all empty
     assert b(1, [(0, 1, 0, 0, 0, 0, 1, 64)], None) == 1                 # null pointers
+    assert b(1, [(0, 1, 0, 0, 0, 0, 1 << 40, 1 << 30)], None) == 2      # size overflow
+    assert b(1, [(2, 1, 0, 0, 0, 0, -1, 64)], None) == 2                # rows < 0
+    assert b(1, [(5, 1, 0, 0, 0, 0, -1, 64)], None) == 1                # bad kind beats bad shape
+    ef = mxq.mxq_exp_free_quantize
+    assert ef(None, 0, 64, None, None, None) == 0
+    assert ef(None, 2, 40, None, None, None) == 2
+    assert ef(None, 1, 64, None, None, None) == 1
+    assert ef(None, 1 << 40, 1 << 20, None, None, None) == 2
+    qc, dc = mxq.mxq_quantize_cols, mxq.mxq_dequantize_cols
+    assert qc(1, None, 1, 0, 64, None, None, None) == 0
+    assert qc(1, None, 1, 48, 64, None, None, None) == 2                # rows % 32
+    assert qc(1, None, 1, 64, 48, None, None, None) == 2                # cols % 32
+    assert qc(1, None, 1, 1 << 40, 64, None, None, None) == 2           # too many tile rows
+    assert qc(1, None, 1, 64, 64, None, None, None) == 1
+    assert qc(8, None, 1, 64, 64, None, None, None) == 1
+    assert dc(1, None, None, 0, 64, None, 1, None) == 0
+    assert dc(1, None, None, 64, 1 << 50, None, 1, None) == 2
+    assert dc(1, None, None, 64, 64, None, 1, None) == 1
+    qx, dx, fx = mxq.mxq_quantize_exmy, mxq.mxq_dequantize_exmy, mxq.mxq_fake_quantize_exmy
+    assert qx(2, 3, None, 0, 0, 64, None, None, None) == 0
+    assert qx(6, 1, None, 0, 1, 64, None, None, None) == 4              # E > 5
+    assert qx(2, 7, None, 0, 1, 64, None, None, None) == 4              # W = 10
+    assert qx(1, 0, None, 0, 1, 64, None, None, None) == 4              # M = 0
+    assert qx(2, 3, None, 4, 1, 64, None, None, None) == 1              # bad dtype
+    assert qx(2, 3, None, 0, 1, 48, None, None, None) == 2
+    assert qx(2, 3, None, 0, 1, 64, None, None, None) == 1
+    assert dx(0, 5, None, None, 0, 64, None, 0, None) == 0
+    assert dx(0, 5, None, None, 1, 64, None, 0, None) == 1
+    assert fx(5, 3, None, 1, 1 << 40, 1 << 20, None, None) == 2
+    assert fx(5, 3, None, 1, 1, 64, None, None) == 1
     assert mxq.mxq_selftest_timeout(0) == 1 and mxq.mxq_selftest_timeout(1001) == 1
     for s in range(7):
         assert mxq.mxq_status_string(s)
