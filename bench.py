@@ -13,7 +13,10 @@ timed K steps are one CUDA graph (one kernel node per step, nothing between
 them), uploaded to the device first (cudaGraphUpload: a one-time setup that
 would otherwise fall inside the timed replay), then replayed once between CUDA
 events on the launching stream; clocks and
-throttle reasons are sampled through NVML while it runs. The roofline's
+throttle reasons are sampled through NVML (the CUDA device found by its UUID)
+while it runs, and a replay that saw a thermal or hardware slowdown, or a clock
+stuck well below the maximum with no reason given, is taken once more (all
+ranks alike; the dropped one is listed under clocks.rejected_runs). The roofline's
 kernel is the batch kernel: the timed region launches nothing else, so its
 average launch duration is that region's device time / K. per_op: the four
 single-operation kernels, each timed as a graph of K launches of it alone. e2e: the same step through the public Python API from pinned host
@@ -101,20 +104,36 @@ class ClockSampler:
         "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
     }
 
-    def __init__(self, index, period=0.002):
+    # a timed region that saw one of these is not kept
+    REJECT = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+    def __init__(self, index, period=0.002, uuid=None):
         self.samples = []
         self.period = period
         self.ok = False
+        self.match = None
         try:
             import pynvml
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.h, self.match = self.handle(pynvml, index, uuid)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
             self.ok = True
         except Exception as e:  # no NVML: report it, never guess
             self.err = str(e)
         self._stop = threading.Event()
+
+    @staticmethod
+    def handle(nv, index, uuid):
+        """NVML numbers every GPU of the machine, CUDA only the visible ones: find the CUDA
+        device by its UUID, and by index only when that fails."""
+        if uuid:
+            u = str(uuid)
+            try:
+                return nv.nvmlDeviceGetHandleByUUID(u if u.startswith("GPU-") else "GPU-" + u), "uuid"
+            except Exception:
+                pass
+        return nv.nvmlDeviceGetHandleByIndex(index), "index"
 
     def _run(self):
         nv = self.nv
@@ -154,7 +173,17 @@ class ClockSampler:
                 if r & bit:
                     seen.add(name)
         return {"sm_mhz": statistics.median(mhz) if mhz[0] is not None else None, "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(seen), "samples": len(self.samples)}
+                "reasons": sorted(seen), "samples": len(self.samples), "nvml_device": self.match}
+
+    @classmethod
+    def rejected(cls, summary):
+        """True for a region that saw a thermal or hardware slowdown, or whose median SM clock
+        sat well below the maximum with no reason given (a clock lock left by someone else)."""
+        reasons = summary.get("reasons") or []
+        if any(r in cls.REJECT for r in reasons):
+            return True
+        mhz, top = summary.get("sm_mhz"), summary.get("sm_max_mhz")
+        return bool(mhz and top and mhz < 0.9 * top and not reasons)
 
 
 # ---- the oracle as CPU baseline / reference arm -----------------------------------------
@@ -223,6 +252,37 @@ def max_over_ranks(value, dist, device):
 def job_gbs(world, bytes_per_step, steps, ms_total_max):
     """Whole-job throughput: every rank moved bytes_per_step * steps; time = slowest rank."""
     return world * bytes_per_step * steps / (ms_total_max * 1e-3) / 1e9
+
+
+def timed_replay(torch, graph, device, dist, sampler, attempts=2):
+    """Device time (ms) of one replay of `graph` between CUDA events on the current stream,
+    with the clocks sampled while it runs. A replay whose clock record is rejected
+    (ClockSampler.rejected) on any rank is taken again, up to `attempts` in all; every rank
+    takes the same number, since the decision is a max over ranks. Returns (ms, clocks) of the
+    last replay; clocks lists the rejected ones under "rejected_runs"."""
+    multi = dist is not None and dist.is_initialized() and dist.get_world_size() > 1
+    rejected = []
+    for attempt in range(attempts):
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        if multi:
+            dist.barrier()
+        torch.cuda.synchronize()
+        with sampler() as clk:
+            start.record()
+            graph.replay()
+            end.record()
+            torch.cuda.synchronize()
+        if multi:
+            dist.barrier()
+        ms, clocks = start.elapsed_time(end), clk.summary()
+        mine = ClockSampler.rejected(clocks)
+        bad = max_over_ranks(1.0 if mine else 0.0, dist if multi else None, device)
+        if bad == 0.0 or attempt == attempts - 1:
+            if rejected:
+                clocks["rejected_runs"] = rejected
+            return ms, clocks
+        rejected.append({"ms": round(ms, 4), "clocks": clocks, "on": "this rank" if mine else "another rank"})
 
 
 # ---- the GPU arm --------------------------------------------------------------------------
@@ -576,19 +636,9 @@ def main():
     gt = graph_of(torch, [step_batch(mxq, sets, k) for k in range(args.warmup, args.warmup + args.steps)])
     uploaded = upload_graph(torch, gt)
     torch.cuda.synchronize()
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        start.record()
-        gt.replay()
-        end.record()
-        torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    ms_total = start.elapsed_time(end)
+    uuid = getattr(torch.cuda.get_device_properties(local), "uuid", None)
+    ms_total, clocks = timed_replay(torch, gt, "cuda", dist if world > 1 else None,
+                                    lambda: ClockSampler(local, uuid=uuid))
     del gt, gw
     # the single-operation kernels, for comparison: K back-to-back launches of one (same rotation, cold data)
     op_ms = {}
@@ -621,7 +671,7 @@ def main():
         "roofline": {"bound": "hbm", "kernel": "k_batch (4 conversions per launch)", "achieved": round(ach, 1),
                      "peak": hbm, "peak_source": how, "unit": "GB/s", "frac": round(ach / hbm, 4),
                      "traffic": ncu_traffic("batch_step"), "algorithmic_bytes_per_launch": step_bytes},
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "gpu_launches": args.steps,
     }
     if rank == 0:

@@ -1,0 +1,211 @@
+"""Host logic of bench.py's timed region, on CPU with fakes: the NVML device is found by the
+CUDA device's UUID (NVML numbers every GPU of the machine, CUDA only the visible ones), the
+clock-event reasons are decoded from their bit mask, a region that saw a thermal or hardware
+slowdown (or a median clock well below the maximum with no reason) is rejected and taken once
+more, and with two gloo ranks both take the same number of replays when only one rank's record
+is rejected."""
+import os
+import socket
+import sys
+import types
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def fake_nvml(uuids, mhz=1965, reasons=0, max_mhz=1965):
+    """A stand-in for pynvml: device i has UUID uuids[i]; the clock and reasons are read from
+    the module's attributes, so a test can change them while a sampler runs."""
+    nv = types.SimpleNamespace(NVML_CLOCK_SM=1, mhz=mhz, reasons=reasons, inits=0)
+
+    class NVMLError(Exception):
+        pass
+
+    def by_uuid(u):
+        if u not in uuids:
+            raise NVMLError("not found")
+        return ("dev", uuids.index(u))
+
+    def by_index(i):
+        if not 0 <= i < len(uuids):
+            raise NVMLError("bad index")
+        return ("dev", i)
+
+    def init():
+        nv.inits += 1
+
+    nv.nvmlInit = init
+    nv.nvmlDeviceGetHandleByUUID = by_uuid
+    nv.nvmlDeviceGetHandleByIndex = by_index
+    nv.nvmlDeviceGetMaxClockInfo = lambda h, kind: max_mhz
+    nv.nvmlDeviceGetClockInfo = lambda h, kind: nv.mhz
+    nv.nvmlDeviceGetCurrentClocksEventReasons = lambda h: nv.reasons
+    return nv
+
+
+def test_nvml_device_found_by_uuid(monkeypatch):
+    nv = fake_nvml(["GPU-aaaa", "GPU-bbbb", "GPU-cccc"])
+    monkeypatch.setitem(sys.modules, "pynvml", nv)
+    s = bench.ClockSampler(0, uuid="bbbb")  # CUDA device 0 is the machine's GPU 1
+    assert s.ok and s.h == ("dev", 1) and s.match == "uuid"
+    s = bench.ClockSampler(0, uuid="GPU-cccc")
+    assert s.h == ("dev", 2) and s.match == "uuid"
+    s = bench.ClockSampler(1, uuid="dddd")  # unknown UUID: the index
+    assert s.h == ("dev", 1) and s.match == "index"
+    s = bench.ClockSampler(2)
+    assert s.h == ("dev", 2) and s.match == "index"
+
+
+def test_no_nvml_is_reported_not_guessed(monkeypatch):
+    monkeypatch.setitem(sys.modules, "pynvml", None)  # import fails
+    s = bench.ClockSampler(0)
+    with s:
+        pass
+    assert not s.ok
+    assert s.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+
+
+def test_sampler_decodes_reasons(monkeypatch):
+    nv = fake_nvml(["GPU-aaaa"], mhz=1800, reasons=0x4 | 0x40)  # sw_power_cap + hw_thermal_slowdown
+    monkeypatch.setitem(sys.modules, "pynvml", nv)
+    with bench.ClockSampler(0, period=0.001, uuid="aaaa") as s:
+        import time
+        time.sleep(0.02)
+    sm = s.summary()
+    assert sm["sm_mhz"] == 1800 and sm["sm_max_mhz"] == 1965 and sm["samples"] >= 2
+    assert sm["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert sm["nvml_device"] == "uuid"
+    assert bench.ClockSampler.rejected(sm)
+
+
+@pytest.mark.parametrize("summary,bad", [
+    ({"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}, False),
+    ({"sm_mhz": 1300, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"]}, False),  # kept and noted
+    ({"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": ["hw_slowdown"]}, True),
+    ({"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": ["sw_thermal_slowdown"]}, True),
+    ({"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": ["gpu_idle", "hw_thermal_slowdown"]}, True),
+    ({"sm_mhz": 1200, "sm_max_mhz": 1965, "reasons": []}, True),  # stuck low, no reason: a lock
+    ({"sm_mhz": 1800, "sm_max_mhz": 1965, "reasons": []}, False),
+    ({"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}, False),
+])
+def test_rejection_rule(summary, bad):
+    assert bench.ClockSampler.rejected(summary) is bad
+
+
+class FakeTorch:
+    """torch.cuda's events and synchronize over a fake device clock that graph replays advance."""
+
+    def __init__(self):
+        self.now = 0.0
+        self.syncs = 0
+        fake = self
+
+        class Event:
+            def __init__(self, enable_timing=False):
+                assert enable_timing
+                self.at = None
+
+            def record(self):
+                self.at = fake.now
+
+            def elapsed_time(self, other):
+                return other.at - self.at
+
+        def synchronize():
+            fake.syncs += 1
+
+        self.cuda = types.SimpleNamespace(Event=Event, synchronize=synchronize)
+
+
+class FakeGraph:
+    def __init__(self, t, durations):
+        self.t, self.durations, self.replays = t, list(durations), 0
+
+    def replay(self):
+        self.t.now += self.durations[self.replays]
+        self.replays += 1
+
+
+def sampler_sequence(summaries):
+    it = iter(summaries)
+
+    class S:
+        def __enter__(self):
+            self.s = next(it)
+            return self
+
+        def __exit__(self, *a):
+            return False
+
+        def summary(self):
+            return dict(self.s)
+
+    return S
+
+
+GOOD = {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}
+HOT = {"sm_mhz": 1600, "sm_max_mhz": 1965, "reasons": ["hw_thermal_slowdown"]}
+
+
+def test_timed_replay_keeps_a_clean_region():
+    t = FakeTorch()
+    g = FakeGraph(t, [12.5, 99.0])
+    ms, clocks = bench.timed_replay(t, g, "cpu", None, sampler_sequence([GOOD, GOOD]))
+    assert ms == 12.5 and g.replays == 1 and clocks == GOOD
+
+
+def test_timed_replay_retakes_a_rejected_region_once():
+    t = FakeTorch()
+    g = FakeGraph(t, [20.0, 12.5, 99.0])
+    ms, clocks = bench.timed_replay(t, g, "cpu", None, sampler_sequence([HOT, GOOD, GOOD]))
+    assert ms == 12.5 and g.replays == 2
+    assert clocks["reasons"] == []
+    assert clocks["rejected_runs"] == [{"ms": 20.0, "clocks": HOT, "on": "this rank"}]
+    # rejected twice: the second is reported as it is, with its reasons, for the reader to judge
+    t = FakeTorch()
+    g = FakeGraph(t, [20.0, 21.0, 99.0])
+    ms, clocks = bench.timed_replay(t, g, "cpu", None, sampler_sequence([HOT, HOT, GOOD]))
+    assert ms == 21.0 and g.replays == 2 and clocks["reasons"] == ["hw_thermal_slowdown"]
+    assert len(clocks["rejected_runs"]) == 1
+
+
+def free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, q):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench as b
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        t = FakeTorch()
+        g = FakeGraph(t, [10.0 + rank, 11.0 + rank, 99.0])
+        seq = [GOOD, GOOD] if rank == 0 else [HOT, GOOD]  # only rank 1 saw a slowdown
+        ms, clocks = b.timed_replay(t, g, "cpu", dist, sampler_sequence(seq))
+        q.put((rank, g.replays, ms, [r["on"] for r in clocks.get("rejected_runs", [])]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ranks_agree_on_a_retake_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=5) for _ in range(2))
+    # both ranks replay twice (same collective steps on every rank) and keep the second replay;
+    # rank 0's clean first replay is dropped because rank 1's was rejected
+    assert got == [(0, 2, 11.0, ["another rank"]), (1, 2, 12.0, ["this rank"])]
