@@ -46,6 +46,7 @@ import synthetic  # noqa: E402
 METRIC = "quantize/fake-quant GB/s (bytes in+out) and % of B200 HBM peak, per format"
 WORKLOAD = "mxfp6_e2m3+e3m2 quantize+dequantize, bf16 4096x4096 weight N(0,0.02) with 0.1% outliers x50, seed 1"
 FALLBACK_HBM = 6650.0
+NOMINAL_HBM = 8000.0  # B200 HBM3e, nominal GB/s (context only; fractions are of the measured copy peak)
 
 
 def peaks():
@@ -668,8 +669,10 @@ def main():
         "frac_hbm": round(value / world / hbm, 4),
         "per_op": {nm: {"ms": round(v, 5), "GB/s": round(op_bytes / (v * 1e-3) / 1e9, 1),
                         "frac_hbm": round(op_bytes / (v * 1e-3) / 1e9 / hbm, 4)} for nm, v in op_ms.items()},
+        "gelem_per_s": round(world * 4 * n * args.steps / (ms_total * 1e-3) / 1e9, 2),
         "roofline": {"bound": "hbm", "kernel": "k_batch (4 conversions per launch)", "achieved": round(ach, 1),
                      "peak": hbm, "peak_source": how, "unit": "GB/s", "frac": round(ach / hbm, 4),
+                     "peak_nominal": NOMINAL_HBM, "frac_nominal": round(ach / NOMINAL_HBM, 4),
                      "traffic": ncu_traffic("batch_step"), "algorithmic_bytes_per_launch": step_bytes},
         "clocks": clocks,
         "gpu_launches": args.steps,

@@ -88,6 +88,34 @@ def test_tables_monotone_and_round_trip(fmt):
         assert oracle.round_mag(fmt, pos[c]) == c
 
 
+@pytest.mark.parametrize("fmt", ALL_FORMATS)
+def test_codes_round_trip_through_blocks_at_extreme_scales(fmt):
+    """Every non-NaN code c, of either sign, written as the fp32 value decode(c)·2^k into blocks
+    that also hold the largest code (so the block maximum fixes the scale at exactly 2^k), comes
+    back as c with scale byte k + 127 for k in {-127, -20, 0, 20, 127 - emax}: the ends of the
+    E8M0 range, where a wrong clamp or an fp32 subnormal input would show; and the dequantized
+    values are the inputs, bit for bit."""
+    w = oracle.bits(fmt)
+    t = oracle.decode_table(fmt)
+    codes = np.array([c for c in range(1 << w) if not np.isnan(t[c])], dtype=np.uint32)
+    top = int(np.argmax(np.where(np.isnan(t), -np.inf, t)))  # the largest positive code
+    nblocks = -(-codes.size // 31)
+    want = np.full((nblocks, 32), top, dtype=np.uint32)
+    want[:, 1:].flat[:codes.size] = codes
+    for k in [-127, -20, 0, 20, 127 - oracle.emax(fmt)]:
+        v = t[want] * 2.0 ** k
+        x = v.astype(np.float32)
+        assert np.array_equal(x.astype(np.float64), v)  # every value is an fp32 number
+        got_codes, scales = oracle.quantize(x, fmt)
+        bytes_ = (scales & 0xFF) if fmt == "axs6" else scales
+        assert np.all(bytes_ == k + 127), (fmt, k)
+        P = oracle.payload_bytes(fmt)
+        for b in range(nblocks):
+            assert np.array_equal(oracle.unpack_codes(got_codes[b, :P], fmt), want[b]), (fmt, k, b)
+        back = oracle.dequantize(got_codes, scales, fmt, x.shape, "f32")
+        assert np.array_equal(back.view(np.uint32), x.view(np.uint32)), (fmt, k)
+
+
 def test_max_values_and_emax():
     expect = {"axs6": (31 / 16, 0), "mxfp6_e2m3": (7.5, 2), "mxfp6_e3m2": (28.0, 4),
               "mxfp8": (448.0, 8), "mxfp4": (6.0, 2)}
