@@ -231,6 +231,27 @@ def test_round_matches_library_cast(fmt):
         assert np.array_equal(ours, tc)
 
 
+@pytest.mark.parametrize("fmt", ALL_FORMATS)
+def test_round_ten_million_fp32_patterns(fmt):
+    """10^7 fp32 bit patterns drawn uniformly between those of 2^-14 and 2·max (every binade
+    of the grid and its subnormal range, all 23 mantissa bits random): the oracle's rounding
+    equals the library's round-to-nearest-even cast after clamping (ml_dtypes for the OCP
+    formats; for AXS-6, whose element is the fixed-point m/16, numpy's rint of 16·y)."""
+    rng = np.random.default_rng(2024)
+    mx = oracle.maxval(fmt)
+    lo = np.array([2.0 ** -14], dtype=np.float32).view(np.uint32)[0]
+    hi = np.array([2 * mx], dtype=np.float32).view(np.uint32)[0]
+    y = rng.integers(lo, hi, 10_000_000, dtype=np.uint32).view(np.float32)
+    yc = np.minimum(y, np.float32(mx))
+    if fmt == "axs6":
+        lib_codes = np.rint(yc.astype(np.float64) * 16).astype(np.uint32)
+    else:
+        lib_codes = yc.astype(ML[fmt]).view(np.uint8).astype(np.uint32)
+    ours = oracle.round_mags(fmt, y.astype(np.float64))
+    bad = np.flatnonzero(ours != lib_codes)
+    assert bad.size == 0, (fmt, y[bad[:5]], ours[bad[:5]], lib_codes[bad[:5]])
+
+
 # ---- the block: scale rule, signs, specials -----------------------------------------
 
 def oracle_block_bruteforce(fmt, x):
