@@ -590,7 +590,7 @@ def main():
                     help="run one kernel a few times on its workload and exit (for ncu captures)")
     ap.add_argument("--profile-reps", type=int, default=3)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--steps", type=int, default=1600)
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", default="mxq", choices=["mxq", "reference"])
     ap.add_argument("--ref-seconds", type=float, default=20.0)

@@ -116,12 +116,13 @@ def test_config4_gradients_fake_quantize():
 
 
 def test_config5_exp_quantize_mxfp4():
+    """All 4096 rows (134M scores, each through the method's own fp32 exponential) against
+    the oracle, bit for bit: about ten seconds of oracle time."""
     s = synthetic.attention_scores(seed=4)
     codes, scales = mxq.exp_quantize(dev(s), "mxfp4")
-    rows = sample(s.shape[0], 48, 3)
-    oc, os_ = oracle.exp_quantize(s[rows], "mxfp4")
-    assert np.array_equal(host(scales)[rows], os_)
-    assert np.array_equal(host(codes)[rows], oc)
+    oc, os_ = oracle.exp_quantize(s, "mxfp4")
+    assert np.array_equal(host(scales), os_)
+    assert np.array_equal(host(codes), oc)
     # every row's maximum key: p = 1 -> scale byte 125, E2M1 code 0x6; no sign bits
     hc, hs = host(codes), host(scales)
     j = np.argmax(s, axis=1)
