@@ -3,9 +3,12 @@
 The functions named like the C entry points (mxq_quantize, ...) take raw
 integers (device pointers, sizes, a cudaStream_t handle) and return the
 mxq_status code. The torch-facing helpers below them (quantize, dequantize,
-fake_quantize, exp_quantize, exp_free_quantize, quantize_grouped) only allocate outputs with
-torch, read pointers/strides and the current stream, call the C entry point
-and raise MXQError on a non-zero status. Every step of the method runs in the
+fake_quantize, exp_quantize, exp_free_quantize, quantize_grouped, batch, ...)
+only allocate outputs with torch, refuse host tensors and caller-supplied
+buffers that are non-contiguous or smaller than the shape needs (the C calls
+take bare pointers, so a short buffer would be read or written past its end),
+read pointers and the current stream, call the C entry point and raise MXQError
+on a non-zero status. Every step of the method runs in the
 CUDA kernels of libmxq; there is no CPU path: if libmxq.so is missing, every
 call raises.
 """
@@ -242,6 +245,32 @@ def _check(status, what):
         raise MXQError(status, what)
 
 
+def _on_gpu(t, what):
+    """The library computes on the GPU only: a host tensor is refused here, before any call."""
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor (libmxq has no CPU path)")
+
+
+def _fits(t, nbytes, what):
+    """A buffer handed to the library as a bare pointer must be contiguous and hold at least
+    nbytes, or a kernel would read or write past the tensor's end."""
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    have = t.numel() * t.element_size()
+    if have < nbytes:
+        raise ValueError(f"{what} holds {have} bytes, the call needs {nbytes}")
+
+
+def _nblocks(rows, cols):
+    return rows * (cols // 32) if rows >= 0 and cols > 0 else 0
+
+
+def _codes_scales_bytes(fmt, rows, cols):
+    """Bytes of the code and scale arrays (0 for a shape the library rejects)."""
+    f = _fmt(fmt)
+    return mxq_codes_bytes(f, rows, cols), mxq_scales_bytes(f, rows, cols)
+
+
 def scale_dtype(fmt):
     torch = _torch()
     return torch.int16 if fmt == "axs6" else torch.uint8
@@ -261,11 +290,15 @@ def quantize(x, fmt, codes=None, scales=None, stream=None):
     """x [..., cols] (bf16/fp32, contiguous, CUDA) -> (codes uint8 [rows, cols/32*P], scales)."""
     if not x.is_contiguous():
         raise ValueError("x must be contiguous")
+    _on_gpu(x, "x")
     rows, cols = _as2d(x)
+    nc, ns = _codes_scales_bytes(fmt, rows, cols)
     if codes is None:
         codes = empty_codes(fmt, rows, cols, x.device)
     if scales is None:
         scales = empty_scales(fmt, rows, cols, x.device)
+    _fits(codes, nc, "codes")
+    _fits(scales, ns, "scales")
     _check(mxq_quantize(_fmt(fmt), x.data_ptr(), _dt(x), rows, cols, codes.data_ptr(), scales.data_ptr(),
                         _stream(stream)), "mxq_quantize")
     return codes, scales
@@ -274,12 +307,24 @@ def quantize(x, fmt, codes=None, scales=None, stream=None):
 def dequantize(codes, scales, fmt, shape, dtype=None, out=None, stream=None):
     """codes + scales -> values of `shape` (last dim = cols) and `dtype` (default bf16)."""
     torch = _torch()
+    _on_gpu(codes, "codes")
     if out is None:
         out = torch.empty(tuple(shape), dtype=dtype or torch.bfloat16, device=codes.device)
     rows, cols = _as2d(out)
+    nc, ns = _codes_scales_bytes(fmt, rows, cols)
+    _fits(codes, nc, "codes")
+    _fits(scales, ns, "scales")
+    _fits(out, 0, "out")
     _check(mxq_dequantize(_fmt(fmt), codes.data_ptr(), scales.data_ptr(), rows, cols, out.data_ptr(), _dt(out),
                           _stream(stream)), "mxq_dequantize")
     return out
+
+
+def _same_values(x, out):
+    """out of a fake-quantize: x's type and element count, contiguous."""
+    if out.dtype != x.dtype or out.numel() != x.numel():
+        raise ValueError(f"out must have x's dtype and size ({x.dtype}, {x.numel()}), got ({out.dtype}, {out.numel()})")
+    _fits(out, 0, "out")
 
 
 def fake_quantize(x, fmt="axs6", block_size=32, out=None, stream=None):
@@ -289,8 +334,10 @@ def fake_quantize(x, fmt="axs6", block_size=32, out=None, stream=None):
     torch = _torch()
     if not x.is_contiguous():
         raise ValueError("x must be contiguous")
+    _on_gpu(x, "x")
     if out is None:
         out = torch.empty_like(x)
+    _same_values(x, out)
     rows, cols = _as2d(x)
     _check(mxq_fake_quantize(_fmt(fmt), x.data_ptr(), _dt(x), rows, cols, out.data_ptr(), _stream(stream)),
            "mxq_fake_quantize")
@@ -302,11 +349,15 @@ def exp_quantize(scores, fmt="mxfp4", codes=None, scales=None, stream=None):
     torch = _torch()
     if scores.dtype != torch.float32 or not scores.is_contiguous():
         raise ValueError("scores must be contiguous float32")
+    _on_gpu(scores, "scores")
     rows, cols = _as2d(scores)
+    nc, ns = _codes_scales_bytes(fmt, rows, cols)
     if codes is None:
         codes = empty_codes(fmt, rows, cols, scores.device)
     if scales is None:
         scales = empty_scales(fmt, rows, cols, scores.device)
+    _fits(codes, nc, "codes")
+    _fits(scales, ns, "scales")
     _check(mxq_exp_quantize(_fmt(fmt), scores.data_ptr(), rows, cols, codes.data_ptr(), scales.data_ptr(),
                             _stream(stream)), "mxq_exp_quantize")
     return codes, scales
@@ -318,11 +369,15 @@ def exp_free_quantize(scores, codes=None, scales=None, stream=None):
     torch = _torch()
     if scores.dtype != torch.float32 or not scores.is_contiguous():
         raise ValueError("scores must be contiguous float32")
+    _on_gpu(scores, "scores")
     rows, cols = _as2d(scores)
+    nc, ns = _codes_scales_bytes("mxfp4", rows, cols)
     if codes is None:
         codes = empty_codes("mxfp4", rows, cols, scores.device)
     if scales is None:
         scales = empty_scales("mxfp4", rows, cols, scores.device)
+    _fits(codes, nc, "codes")
+    _fits(scales, ns, "scales")
     _check(mxq_exp_free_quantize(scores.data_ptr(), rows, cols, codes.data_ptr(), scales.data_ptr(), _stream(stream)),
            "mxq_exp_free_quantize")
     return codes, scales
@@ -334,11 +389,15 @@ def quantize_mma(x, fmt, codes=None, scales=None, stream=None):
     torch = _torch()
     if not x.is_contiguous():
         raise ValueError("x must be contiguous")
+    _on_gpu(x, "x")
     rows, cols = _as2d(x)
+    nc, _ = _codes_scales_bytes(fmt, rows, cols)
     if codes is None:
         codes = empty_codes(fmt, rows, cols, x.device)
     if scales is None:
         scales = torch.empty(mxq_mma_scales_bytes(rows, cols), dtype=torch.uint8, device=x.device)
+    _fits(codes, nc, "codes")
+    _fits(scales, mxq_mma_scales_bytes(rows, cols), "scales")
     _check(mxq_quantize_mma(_fmt(fmt), x.data_ptr(), _dt(x), rows, cols, codes.data_ptr(), scales.data_ptr(),
                             _stream(stream)), "mxq_quantize_mma")
     return codes, scales
@@ -349,9 +408,11 @@ def swizzle_scales(scales, out=None, stream=None):
     torch = _torch()
     if scales.dtype != torch.uint8 or scales.dim() != 2 or not scales.is_contiguous():
         raise ValueError("scales must be a contiguous 2-D uint8 tensor")
+    _on_gpu(scales, "scales")
     rows, kb = scales.shape
     if out is None:
         out = torch.empty(mxq_mma_scales_bytes(rows, 32 * kb), dtype=torch.uint8, device=scales.device)
+    _fits(out, mxq_mma_scales_bytes(rows, 32 * kb), "out")
     _check(mxq_swizzle_scales(scales.data_ptr(), rows, kb, out.data_ptr(), _stream(stream)), "mxq_swizzle_scales")
     return out
 
@@ -381,11 +442,18 @@ def batch(ops, stream=None):
             raise ValueError(f"unknown batch op {kind!r}")
         if not vals.is_contiguous():
             raise ValueError("value tensors must be contiguous")
+        _on_gpu(vals, "batch values")
         if dtype is None:
             dtype = _dt(vals)
         elif _dt(vals) != dtype:
             raise TypeError("all values of a batch must have one dtype")
         rows, cols = _as2d(vals)
+        if kind == "fake_quantize":
+            _same_values(x, out)
+        else:
+            nc, ns = _codes_scales_bytes(fmt, rows, cols)
+            _fits(codes, nc, "codes")
+            _fits(scales, ns, "scales")
         descs.append((OP_KINDS[kind], _fmt(fmt), *d, rows, cols))
     if not descs:
         raise ValueError("empty batch")
@@ -404,11 +472,17 @@ def quantize_grouped(xs, fmt, outs=None, stream=None):
         for x in xs:
             r, c = _as2d(x)
             outs.append((empty_codes(fmt, r, c, x.device), empty_scales(fmt, r, c, x.device)))
+    if len(outs) != len(xs):
+        raise ValueError("one (codes, scales) pair per tensor")
     descs = []
     for x, (c, s) in zip(xs, outs):
         if _dt(x) != dt or not x.is_contiguous():
             raise ValueError("grouped tensors must be contiguous and share one dtype")
+        _on_gpu(x, "grouped tensors")
         r, k = _as2d(x)
+        nc, ns = _codes_scales_bytes(fmt, r, k)
+        _fits(c, nc, "codes")
+        _fits(s, ns, "scales")
         descs.append((x.data_ptr(), c.data_ptr(), s.data_ptr(), r, k))
     _check(mxq_quantize_grouped(_fmt(fmt), dt, descs, _stream(stream)), "mxq_quantize_grouped")
     return outs
@@ -419,11 +493,15 @@ def quantize_cols(x, fmt, codes=None, scales=None, stream=None):
     codes [cols, rows/32*P], scales [cols, rows/32]."""
     if not x.is_contiguous() or x.dim() != 2:
         raise ValueError("x must be a contiguous 2-D tensor")
+    _on_gpu(x, "x")
     rows, cols = x.shape
+    nc, ns = _codes_scales_bytes(fmt, cols, rows)
     if codes is None:
         codes = empty_codes(fmt, cols, rows, x.device)
     if scales is None:
         scales = empty_scales(fmt, cols, rows, x.device)
+    _fits(codes, nc, "codes")
+    _fits(scales, ns, "scales")
     _check(mxq_quantize_cols(_fmt(fmt), x.data_ptr(), _dt(x), rows, cols, codes.data_ptr(), scales.data_ptr(),
                              _stream(stream)), "mxq_quantize_cols")
     return codes, scales
@@ -432,9 +510,16 @@ def quantize_cols(x, fmt, codes=None, scales=None, stream=None):
 def dequantize_cols(codes, scales, fmt, shape, dtype=None, out=None, stream=None):
     """Inverse of quantize_cols: values of `shape` = (rows, cols)."""
     torch = _torch()
+    _on_gpu(codes, "codes")
     if out is None:
         out = torch.empty(tuple(shape), dtype=dtype or torch.bfloat16, device=codes.device)
+    if out.dim() != 2:
+        raise ValueError("out must be 2-D (rows, cols)")
     rows, cols = out.shape
+    nc, ns = _codes_scales_bytes(fmt, cols, rows)
+    _fits(codes, nc, "codes")
+    _fits(scales, ns, "scales")
+    _fits(out, 0, "out")
     _check(mxq_dequantize_cols(_fmt(fmt), codes.data_ptr(), scales.data_ptr(), rows, cols, out.data_ptr(), _dt(out),
                                _stream(stream)), "mxq_dequantize_cols")
     return out
@@ -445,12 +530,15 @@ def quantize_exmy(x, ebits, mbits, codes=None, scales=None, stream=None):
     torch = _torch()
     if not x.is_contiguous():
         raise ValueError("x must be contiguous")
+    _on_gpu(x, "x")
     rows, cols = _as2d(x)
     W = 1 + ebits + mbits
     if codes is None:
         codes = torch.empty((rows, (cols // 32) * 4 * W), dtype=torch.uint8, device=x.device)
     if scales is None:
         scales = torch.empty((rows, cols // 32), dtype=torch.uint8, device=x.device)
+    _fits(codes, _nblocks(rows, cols) * 4 * max(W, 0), "codes")
+    _fits(scales, _nblocks(rows, cols), "scales")
     _check(mxq_quantize_exmy(ebits, mbits, x.data_ptr(), _dt(x), rows, cols, codes.data_ptr(), scales.data_ptr(),
                              _stream(stream)), "mxq_quantize_exmy")
     return codes, scales
@@ -458,9 +546,13 @@ def quantize_exmy(x, ebits, mbits, codes=None, scales=None, stream=None):
 
 def dequantize_exmy(codes, scales, ebits, mbits, shape, dtype=None, out=None, stream=None):
     torch = _torch()
+    _on_gpu(codes, "codes")
     if out is None:
         out = torch.empty(tuple(shape), dtype=dtype or torch.bfloat16, device=codes.device)
     rows, cols = _as2d(out)
+    _fits(codes, _nblocks(rows, cols) * 4 * max(1 + ebits + mbits, 0), "codes")
+    _fits(scales, _nblocks(rows, cols), "scales")
+    _fits(out, 0, "out")
     _check(mxq_dequantize_exmy(ebits, mbits, codes.data_ptr(), scales.data_ptr(), rows, cols, out.data_ptr(),
                                _dt(out), _stream(stream)), "mxq_dequantize_exmy")
     return out
@@ -470,8 +562,10 @@ def fake_quantize_exmy(x, ebits, mbits, out=None, stream=None):
     torch = _torch()
     if not x.is_contiguous():
         raise ValueError("x must be contiguous")
+    _on_gpu(x, "x")
     if out is None:
         out = torch.empty_like(x)
+    _same_values(x, out)
     rows, cols = _as2d(x)
     _check(mxq_fake_quantize_exmy(ebits, mbits, x.data_ptr(), _dt(x), rows, cols, out.data_ptr(), _stream(stream)),
            "mxq_fake_quantize_exmy")
