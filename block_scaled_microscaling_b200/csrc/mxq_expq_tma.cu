@@ -35,6 +35,7 @@
 // warp has given up): a wait that runs out sets the library's device error
 // word, which mxq_check_device reports as MXQ_ERR_TIMEOUT, and the CTA leaves
 // after the producer has waited (bounded again) for its own copies in flight.
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -546,19 +547,22 @@ cudaError_t launch_selftest_timeout(unsigned long long limit_ns, cudaStream_t st
     return cudaGetLastError();
 }
 
-// address of the device error word on the current device (cached per device)
+// address of the device error word on the current device (cached per device; calls may come
+// from several host threads at once, so the cache entries are atomic)
 cudaError_t device_error_word(unsigned int** p) {
-    static unsigned int* addr[64] = {};
+    static std::atomic<unsigned int*> addr[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!addr[dev]) {
-        void* a = nullptr;
-        if ((e = cudaGetSymbolAddress(&a, g_device_error)) != cudaSuccess) return e;
-        addr[dev] = static_cast<unsigned int*>(a);
+    unsigned int* a = addr[dev].load(std::memory_order_acquire);
+    if (!a) {
+        void* s = nullptr;
+        if ((e = cudaGetSymbolAddress(&s, g_device_error)) != cudaSuccess) return e;
+        a = static_cast<unsigned int*>(s);
+        addr[dev].store(a, std::memory_order_release);
     }
-    *p = addr[dev];
+    *p = a;
     return cudaSuccess;
 }
 
