@@ -209,3 +209,16 @@ def test_ranks_agree_on_a_retake_gloo():
     # both ranks replay twice (same collective steps on every rank) and keep the second replay;
     # rank 0's clean first replay is dropped because rank 1's was rejected
     assert got == [(0, 2, 11.0, ["another rank"]), (1, 2, 12.0, ["this rank"])]
+
+
+def test_oracle_baseline_on_several_threads():
+    """The CPU baseline runs the oracle on independent row samples in several host threads at
+    once; each thread's samples are its own and the bytes add up over all of them."""
+    import numpy as np
+    w = np.zeros((256, 4096), dtype=np.uint16)  # bf16 bits, four 64-row slices
+    v1, i1 = bench.oracle_throughput(w, budget_s=0.05)
+    v2, i2 = bench.oracle_throughput(w, budget_s=0.05, threads=2)
+    assert i1["threads"] == 1 and i2["threads"] == 2
+    assert v1 > 0 and v2 > 0 and i2["samples"] >= 2
+    assert i2["elements"] == i2["samples"] * 64 * 4096
+    assert 1 <= bench.cpu_threads() <= 32
