@@ -176,14 +176,16 @@ int main(void) {
 """
 
 
-def test_plain_c_caller(L, tmp_path):
-    """The boundary is a C ABI: a C99 program built against include/mxq.h alone (no CUDA headers)
-    links with libmxq.so and calls it. Host-only queries; no kernel runs."""
-    src = tmp_path / "caller.c"
+@pytest.mark.parametrize("compiler,std,ext", [("gcc", "c99", "c"), ("g++", "c++11", "cpp")])
+def test_plain_c_caller(L, tmp_path, compiler, std, ext):
+    """The boundary is a C ABI: a C99 program (and the same source as C++11) built against
+    include/mxq.h alone (no CUDA headers) links with libmxq.so and calls it. Host-only queries;
+    no kernel runs."""
+    src = tmp_path / f"caller.{ext}"
     src.write_text(C_PROGRAM)
     exe = tmp_path / "caller"
     libdir = os.path.dirname(mxq.LIB_PATH)
-    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+    r = subprocess.run([compiler, f"-std={std}", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
                         os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir, "-lmxq",
                         "-Wl,-rpath," + libdir], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
