@@ -469,7 +469,7 @@ def workloads_breakdown(torch, mxq, hbm):
     def rec(name, b, n, ms):
         gbs = b / (ms * 1e-3) / 1e9
         out[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "Gelem/s": round(n / (ms * 1e-3) / 1e9, 1),
-                     "frac_hbm": round(gbs / hbm, 4), "bytes": int(b)}
+                     "frac_hbm": round(gbs / hbm, 4), "frac_nominal": round(gbs / NOMINAL_HBM, 4), "bytes": int(b)}
 
     # 1: AXS-6 quick-start fp32 128x256 (L2-resident, launch-latency bound)
     x1 = torch.randn(128, 256, device=dev, generator=gen.manual_seed(0))
@@ -698,7 +698,10 @@ def main():
                              + "; per_op: the single-operation kernels, a graph of K launches of one alone"},
         "frac_hbm": round(value / world / hbm, 4),
         "per_op": {nm: {"ms": round(v, 5), "GB/s": round(op_bytes / (v * 1e-3) / 1e9, 1),
-                        "frac_hbm": round(op_bytes / (v * 1e-3) / 1e9 / hbm, 4)} for nm, v in op_ms.items()},
+                        "Gelem/s": round(n / (v * 1e-3) / 1e9, 1),
+                        "frac_hbm": round(op_bytes / (v * 1e-3) / 1e9 / hbm, 4),
+                        "frac_nominal": round(op_bytes / (v * 1e-3) / 1e9 / NOMINAL_HBM, 4)}
+                   for nm, v in op_ms.items()},
         "gelem_per_s": round(world * 4 * n * args.steps / (ms_total * 1e-3) / 1e9, 2),
         "roofline": {"bound": "hbm", "kernel": "k_batch (4 conversions per launch)", "achieved": round(ach, 1),
                      "peak": hbm, "peak_source": how, "unit": "GB/s", "frac": round(ach / hbm, 4),
