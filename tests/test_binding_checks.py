@@ -10,7 +10,15 @@ pass, torch.cuda.current_stream() would raise on this GPU-less host, not a Value
 import pytest
 import torch
 
+from block_scaled_microscaling_b200 import build as mxq_build
 from block_scaled_microscaling_b200 import mxq
+
+
+@pytest.fixture(scope="module", autouse=True)
+def library():
+    # the size checks use the library's host-only size queries
+    mxq_build.build()
+    return mxq.lib()
 
 
 class FakeCuda:
