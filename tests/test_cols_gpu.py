@@ -1,0 +1,126 @@
+"""GPU parity of the column-direction path at sizes where its persistent grid walks several
+tiles per CTA, bit for bit against the oracle.
+
+Column-direction blocks are 32 consecutive rows of one column; the library lays the result out
+as the row-direction quantization of the transpose (codes [cols, rows/32*P], scales
+[cols, rows/32]), so the oracle runs on x.T. The converted operands feed block-scaled GEMMs
+whose K-contiguous operand is the column direction ("Sonar: Online MXFP6", Start a model and
+Current limits).
+
+The quantize kernel cuts the matrix into tiles of 256 rows x 128 bytes and runs a persistent
+grid of (SMs x resident CTAs) CTAs that walk their tiles through two tensor-copy buffers, so a
+shape with more tiles than twice the grid reuses both buffers and flips their barrier phases
+on every CTA. Each test asserts that premise for its shape before comparing.
+"""
+import functools
+import zlib
+
+import numpy as np
+import pytest
+
+import oracle
+
+torch = pytest.importorskip("torch")
+from block_scaled_microscaling_b200 import mxq  # noqa: E402
+
+from test_parity_gpu import bits, dev, hard_values, host, tdtype  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+FMTS = ["axs6", "mxfp6_e2m3", "mxfp6_e3m2", "mxfp8", "mxfp4"]
+TILE_ROWS, TILE_BYTES = 256, 128
+
+
+def tiles(rows, cols, dtype):
+    tc = TILE_BYTES // (4 if dtype == "f32" else 2)
+    return -(-cols // tc) * -(-rows // TILE_ROWS)
+
+
+def assert_walks_several_tiles(rows, cols, dtype):
+    """Two 32 KB tile buffers per CTA leave room for at most 3 CTAs in an SM's 228 KB of shared
+    memory, so the persistent grid has at most 3 x SMs CTAs; more than twice that many tiles
+    means every CTA takes at least two."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert tiles(rows, cols, dtype) >= 2 * (3 * sms), (rows, cols, dtype)
+
+
+@functools.lru_cache(maxsize=1)
+def big_values(rows, cols, dtype, seed):
+    """Per-block random exponents over +-30 binades and a sprinkling of zero, -0, subnormal and
+    NaN / -Inf column blocks (the blocks are 32 rows of a column here), cheap at any size."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((rows // 32, 32, cols), dtype=np.float32)
+    x *= np.exp2(rng.integers(-30, 31, (rows // 32, 1, cols)).astype(np.float32))
+    kind = rng.integers(0, 64, (rows // 32, cols))
+    rb, c = np.nonzero(kind == 0)
+    x[rb, :, c] = 0.0
+    rb, c = np.nonzero(kind == 1)
+    x[rb, :, c] = -0.0
+    rb, c = np.nonzero(kind == 2)
+    x[rb, :, c] *= np.float32(2.0 ** -120)
+    rb, c = np.nonzero(kind == 3)
+    x[rb, c % 32, c] = np.nan
+    rb, c = np.nonzero(kind == 4)
+    x[rb, c % 32, c] = -np.inf
+    x = np.ascontiguousarray(x.reshape(rows, cols))
+    if dtype == "f32":
+        return x
+    return (x.view(np.uint32) >> 16).astype(np.uint16)  # bf16 by truncation: NaN and -Inf stay what they are
+
+
+def check_full(x, fmt, dtype):
+    rows, cols = x.shape
+    codes, scales = mxq.quantize_cols(dev(x), fmt)
+    xt = np.ascontiguousarray(x.T)
+    oc, os_ = oracle.quantize(xt, fmt)
+    assert np.array_equal(host(scales), os_)
+    assert np.array_equal(host(codes), oc)
+    out = mxq.dequantize_cols(codes, scales, fmt, (rows, cols), tdtype(dtype))
+    ref = np.ascontiguousarray(oracle.dequantize(oc, os_, fmt, xt.shape, dtype).T)
+    assert np.array_equal(bits(host(out)), bits(ref))
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_cols_4096x4096_every_tile(fmt, dtype):
+    """4096 x 4096: 1024 bf16 tiles (2048 fp32 tiles) over the persistent grid, compared in full."""
+    rows, cols = 4096, 4096
+    assert_walks_several_tiles(rows, cols, dtype)
+    x = big_values(rows, cols, dtype, seed=zlib.crc32(repr(("c4096", fmt, dtype)).encode()))
+    check_full(x, fmt, dtype)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype,shape", [("bf16", (4192, 4128)), ("f32", (2336, 4160)), ("bf16", (2080, 8224))])
+def test_cols_ragged_multi_tile(fmt, dtype, shape):
+    """rows % 256 != 0 (a last row tile of 3 or 1 row-blocks) and, for bf16, a last column
+    strip of 32 columns, at sizes where the grid still walks several tiles per CTA."""
+    rows, cols = shape
+    assert_walks_several_tiles(rows, cols, dtype)
+    assert rows % TILE_ROWS != 0
+    x = hard_values(cols, rows, dtype, seed=zlib.crc32(repr(("rag", fmt, dtype, shape)).encode()))
+    # hard_values draws its special blocks along the last dim; transposed they become column blocks
+    check_full(np.ascontiguousarray(x.T), fmt, dtype)
+
+
+@pytest.mark.parametrize("fmt", ["mxfp6_e2m3", "mxfp8", "axs6"])
+@pytest.mark.parametrize("dtype,shape", [("f32", (8192, 8192)), ("bf16", (16384, 8192))])
+def test_cols_large_sampled_columns(fmt, dtype, shape):
+    """The sizes the column figures are measured at (fp32 8192x8192: 8192 tiles; bf16
+    16384x8192: 8192 tiles): the whole matrix converted in one launch, then 96 sampled columns
+    (the first and last included) compared in full with the oracle on those columns, and
+    dequantize_cols of the whole result on the same columns."""
+    rows, cols = shape
+    assert_walks_several_tiles(rows, cols, dtype)
+    x = big_values(rows, cols, dtype, seed=zlib.crc32(repr(("big", dtype, shape)).encode()))
+    codes, scales = mxq.quantize_cols(dev(x), fmt)
+    rng = np.random.default_rng(5)
+    sel = np.unique(np.concatenate([rng.choice(cols, 94, replace=False), [0, cols - 1]]))
+    xs = np.ascontiguousarray(x[:, sel].T)
+    oc, os_ = oracle.quantize(xs, fmt)
+    hs, hc = host(scales), host(codes)
+    assert np.array_equal(hs[sel], os_)
+    assert np.array_equal(hc[sel], oc)
+    out = mxq.dequantize_cols(codes, scales, fmt, (rows, cols), tdtype(dtype))
+    ref = oracle.dequantize(oc, os_, fmt, xs.shape, dtype)
+    assert np.array_equal(bits(host(out)[:, sel].T.copy()), bits(ref))

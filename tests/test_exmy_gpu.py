@@ -1,4 +1,6 @@
 """GPU parity for the eXmY formats (integer rounding path) against the oracle, bit for bit."""
+import functools
+
 import numpy as np
 import pytest
 
@@ -80,3 +82,38 @@ def test_bf16_two_values_per_word_path_at_scale(E, M):
     oc, os_ = oracle.quantize_exmy(np.ascontiguousarray(h[sel]), E, M)
     assert np.array_equal(host(scales)[sel], os_)
     assert np.array_equal(host(codes)[sel], oc)
+
+
+@functools.lru_cache(maxsize=1)
+def fp32_wide(rows, cols, seed):
+    """fp32 values with per-block exponents over +-60 binades, zero, -0 and subnormal blocks."""
+    rng = np.random.default_rng(seed)
+    nb = rows * cols // 32
+    x = rng.standard_normal((nb, 32), dtype=np.float32)
+    x *= np.exp2(rng.integers(-60, 61, (nb, 1)).astype(np.float32))
+    kind = rng.integers(0, 32, nb)
+    x[kind == 0] = 0.0
+    x[kind == 1] = -0.0
+    x[kind == 2] *= np.float32(2.0 ** -80)  # fp32 subnormals
+    return x.reshape(rows, cols)
+
+
+@pytest.mark.parametrize("E,M", SPLITS)
+def test_fp32_quantize_dequantize_fake_quantize_at_scale(E, M):
+    """fp32 2048x8192 (524 288 blocks: the persistent fp32 quantize takes several grid-stride
+    passes, the one-pass dequantize and fake-quantize grids 2048 CTAs) converted whole by
+    quantize, dequantize and fake-quantize; 48 sampled rows of each equal the oracle bit for
+    bit."""
+    rows, cols = 2048, 8192
+    x = fp32_wide(rows, cols, 77)
+    t = dev(x)
+    codes, scales = mxq.quantize_exmy(t, E, M)
+    out = mxq.dequantize_exmy(codes, scales, E, M, (rows, cols), torch.float32)
+    fq = mxq.fake_quantize_exmy(t, E, M)
+    sel = np.sort(np.random.default_rng(10 * E + M).choice(rows, 48, replace=False))
+    xs = np.ascontiguousarray(x[sel])
+    oc, os_ = oracle.quantize_exmy(xs, E, M)
+    assert np.array_equal(host(scales)[sel], os_)
+    assert np.array_equal(host(codes)[sel], oc)
+    assert np.array_equal(bits(host(out)[sel]), bits(oracle.dequantize_exmy(oc, os_, E, M, xs.shape, "f32")))
+    assert np.array_equal(bits(host(fq)[sel]), bits(oracle.fake_quantize_exmy(xs, E, M)))
