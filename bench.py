@@ -1,29 +1,35 @@
 """Throughput of libmxq's block-scaled quantization on B200.
 
-Headline workload: MXFP6 E2M3 and E3M2 quantize + dequantize of one bf16
-4096x4096 weight (N(0, 0.02), 0.1% of entries x50, seed 1). One step = the four
-conversions (quantize E2M3, quantize E3M2, dequantize E2M3, dequantize E3M2) in
-one launch of the batch entry point (mxq_run_batch).
-Metric: algorithmic bytes moved (values in + packed codes + scales, or the
-reverse) / device time, GB/s, and the fraction of the measured HBM copy peak.
+Headline workload: online layer-by-layer conversion of a 36-layer bf16 decoder
+weight stack to MXFP6 E2M3 and to AXS-6 (per layer q 4096x2560, k and v
+1024x2560, o 2560x4096, gate and up 9728x2560, down 2560x9728, stored
+[out, in] so the blocks of 32 run along the input dim; N(0, 0.02), drawn on the
+device from seeded generators). One step = the whole stack converted to both
+formats, one layer at a time: for each layer l one grouped launch
+(mxq_quantize_grouped, the layer's seven tensors) to E2M3 and one to AXS-6 of
+layer (l + 18) mod 36, 72 launches. Each launch reads a 202 MB layer (above the
+126 MB L2) last read 18 layers (about 10 GB of traffic) earlier.
+Metric: algorithmic bytes moved (values in + packed codes + scales) / device
+time, GB/s, and the fraction of the measured HBM copy peak.
 
-Timing: 8 rotating buffer sets (~1 GB) so that every launch reads data last
-touched >= 4 steps (>700 MB of traffic) earlier, i.e. from HBM, not L2; the
-timed K steps are one CUDA graph (one kernel node per step, nothing between
-them), uploaded to the device first (cudaGraphUpload: a one-time setup that
-would otherwise fall inside the timed replay), then replayed once between CUDA
-events on the launching stream; clocks and
-throttle reasons are sampled through NVML (the CUDA device found by its UUID)
-while it runs, and a replay that saw a thermal or hardware slowdown, or a clock
-stuck well below the maximum with no reason given, is taken once more (all
-ranks alike; the dropped one is listed under clocks.rejected_runs). The roofline's
-kernel is the batch kernel: the timed region launches nothing else, so its
-average launch duration is that region's device time / K. per_op: the four
-single-operation kernels, each timed as a graph of K launches of it alone. e2e: the same step through the public Python API from pinned host
-memory, host->device copy of the weight and device->host copy of every
-output inside the timed region. cpu_baseline: the CPU oracle on bounded
-row samples of the same workload, on all host threads (and on one, under
-single_thread).
+Timing: the step is one CUDA graph (72 kernel nodes, nothing between them),
+uploaded to the device first (cudaGraphUpload), then replayed K times between
+CUDA events on the launching stream; clocks and throttle reasons are sampled
+through NVML (the CUDA device found by its UUID) while it runs, and a region
+that saw a thermal or hardware slowdown, or a clock stuck well below the
+maximum with no reason given, is taken once more (all ranks alike; the dropped
+one is listed under clocks.rejected_runs). The device status word is checked
+after every timed region: a kernel whose bounded wait ran out leaves partial
+outputs, and then no speed is reported. The roofline's kernel is the grouped
+quantize (its E2M3 and AXS-6 instances): the timed region launches nothing
+else. per_format: each format's 36 launches alone. e2e: one layer per step
+through the public Python API from pinned host memory, the host->device copy
+of its weights and the device->host copy of both formats' codes and scales
+inside the timed region. cpu_baseline: the CPU oracle on row slices of the same
+workload (the workload's own bits, from the counter-based generator), on all
+host threads (and on one, under single_thread). workloads: every other
+workload's ops, each timed alone, including the bf16 4096x4096 weight step
+(MXFP6 E2M3 + E3M2 quantize + dequantize in one batch launch).
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--no-workloads]
 Multi-GPU (torchrun): independent replicas, one per GPU, no collective on the
@@ -45,7 +51,11 @@ sys.path.insert(0, ROOT)
 import synthetic  # noqa: E402
 
 METRIC = "quantize/fake-quant GB/s (bytes in+out) and % of B200 HBM peak, per format"
-WORKLOAD = "mxfp6_e2m3+e3m2 quantize+dequantize, bf16 4096x4096 weight N(0,0.02) with 0.1% outliers x50, seed 1"
+WORKLOAD = ("online layer-by-layer conversion of a 36-layer bf16 decoder weight stack (per layer q 4096x2560, "
+            "k 1024x2560, v 1024x2560, o 2560x4096, gate 9728x2560, up 9728x2560, down 2560x9728, [out, in], "
+            "N(0,0.02), seed 2) to MXFP6 E2M3 and to AXS-6, blocks of 32 along the input dim")
+WEIGHT_WORKLOAD = "mxfp6_e2m3+e3m2 quantize+dequantize, bf16 4096x4096 weight N(0,0.02) with 0.1% outliers x50, seed 1"
+STACK_FORMATS = ("mxfp6_e2m3", "axs6")
 FALLBACK_HBM = 6650.0
 NOMINAL_HBM = 8000.0  # B200 HBM3e, nominal GB/s (context only; fractions are of the measured copy peak)
 
@@ -199,29 +209,43 @@ def cpu_threads():
     return max(1, min(n, 32))
 
 
-def oracle_throughput(w, budget_s=10.0, threads=1):
-    """The CPU oracle on 64-row samples of the headline workload (E2M3 and E3M2 quantize +
-    dequantize of each sample) for about budget_s seconds, on `threads` host threads at once:
-    the oracle's C calls release the GIL and keep no shared state, each thread takes its own
-    samples. Returns (GB/s over all threads, info)."""
+def oracle_pool(n_slices=24, rows=32, seed=2):
+    """Row slices of the decoder stack with the workload's own bits: for each slice a random
+    (layer, tensor, first row), its rows drawn from the counter-based generator at their element
+    offsets. Made once, before any timing."""
+    rng = np.random.default_rng(12345)
+    pool = []
+    for _ in range(n_slices):
+        layer = int(rng.integers(synthetic.N_LAYERS))
+        k = int(rng.integers(len(synthetic.DECODER_LAYER)))
+        _, nrows, cols = synthetic.DECODER_LAYER[k]
+        r0 = int(rng.integers(nrows - rows + 1))
+        v = synthetic.normals(seed, layer * 7 + k, rows * cols, start=r0 * cols) * 0.02
+        pool.append(synthetic.f32_to_bf16_bits(synthetic.to_f32(v)).reshape(rows, cols))
+    return pool
+
+
+def oracle_throughput(pool, budget_s=10.0, threads=1, formats=STACK_FORMATS):
+    """The CPU oracle quantizing the slices of `pool` (bf16 bits) to each of `formats`, round
+    robin, for about budget_s seconds on `threads` host threads at once: the oracle's C calls
+    release the GIL and keep no shared state, each thread takes its own slices. Returns
+    (GB/s of algorithmic bytes over all threads, info)."""
     import oracle
     oracle.lib()  # load once, before the threads start
-    rows = 64
-    nsl = w.shape[0] // rows
     done = [0] * threads
     count = [0] * threads
+    elems = [0] * threads
     t0 = time.perf_counter()
 
     def work(k):
         i = k
         while True:
-            r0 = (i % nsl) * rows
-            xs = np.ascontiguousarray(w[r0:r0 + rows])
-            for fmt in ("mxfp6_e2m3", "mxfp6_e3m2"):
-                c, s = oracle.quantize(xs, fmt)
-                oracle.dequantize(c, s, fmt, xs.shape, "bf16")
-                done[k] += 2 * nbytes_q(fmt, xs.size, 2)
+            xs = pool[i % len(pool)]
+            for fmt in formats:
+                oracle.quantize(xs, fmt)
+                done[k] += nbytes_q(fmt, xs.size, 2)
             count[k] += 1
+            elems[k] += xs.size
             i += threads
             if time.perf_counter() - t0 >= budget_s:
                 break
@@ -235,33 +259,37 @@ def oracle_throughput(w, budget_s=10.0, threads=1):
         for t in ts:
             t.join()
     el = time.perf_counter() - t0
-    n = sum(count)
-    return sum(done) / el / 1e9, {"rows_per_op": rows, "samples": n, "seconds": round(el, 2),
-                                  "elements": int(n * rows * w.shape[1]), "threads": threads}
+    return sum(done) / el / 1e9, {"samples": sum(count), "seconds": round(el, 2), "elements": int(sum(elems)),
+                                  "threads": threads}
+
+
+def stack_step_bytes():
+    """Algorithmic bytes of one step: the whole stack quantized to both formats."""
+    n = sum(r * c for _, r, c in synthetic.DECODER_LAYER) * synthetic.N_LAYERS
+    return sum(nbytes_q(f, n, 2) for f in STACK_FORMATS), n
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
-    w, _ = synthetic.weight_with_outliers(seed=1)
+    pool = oracle_pool()
     nt = cpu_threads()
     per_step = []
     for _ in range(args.warmup):
-        oracle_throughput(w, budget_s=0.2, threads=nt)
+        oracle_throughput(pool, budget_s=0.2, threads=nt)
     for _ in range(args.steps):
-        v, info = oracle_throughput(w, budget_s=max(0.2, args.ref_seconds / max(1, args.steps)), threads=nt)
+        v, info = oracle_throughput(pool, budget_s=max(0.2, args.ref_seconds / max(1, args.steps)), threads=nt)
         per_step.append(v)
     value = statistics.mean(per_step)
-    hbm, how = peaks()
-    step_bytes = 4 * nbytes_q("mxfp6_e2m3", 4096 * 4096, 2)
+    step_bytes, _ = stack_step_bytes()
+    sample = (f"{len(pool)} slices of 32 rows of the stack's tensors (the workload's own bits), each quantized "
+              f"to MXFP6 E2M3 and AXS-6, oracle in C on {nt} host threads, ~{args.ref_seconds:.0f} s in total")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_bytes / (value * 1e9) * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample": f"64-row slices per op, oracle in C, {nt} host threads"},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": nt, "kind": "oracle",
-                         "sample": f"64-row slices of the 4096x4096 weight on {nt} threads, "
-                                   f"~{args.ref_seconds:.0f} s in total"},
+        "config": {"workload": WORKLOAD, "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": nt, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -285,12 +313,13 @@ def job_gbs(world, bytes_per_step, steps, ms_total_max):
     return world * bytes_per_step * steps / (ms_total_max * 1e-3) / 1e9
 
 
-def timed_replay(torch, graph, device, dist, sampler, attempts=2):
-    """Device time (ms) of one replay of `graph` between CUDA events on the current stream,
-    with the clocks sampled while it runs. A replay whose clock record is rejected
-    (ClockSampler.rejected) on any rank is taken again, up to `attempts` in all; every rank
-    takes the same number, since the decision is a max over ranks. Returns (ms, clocks) of the
-    last replay; clocks lists the rejected ones under "rejected_runs"."""
+def timed_replay(torch, graph, device, dist, sampler, attempts=2, replays=1, after=None):
+    """Device time (ms) of `replays` back-to-back replays of `graph` between CUDA events on the
+    current stream, with the clocks sampled while they run. A region whose clock record is
+    rejected (ClockSampler.rejected) on any rank is taken again, up to `attempts` in all; every
+    rank takes the same number, since the decision is a max over ranks. `after` (if given) runs
+    once each region has synchronized (the device status check). Returns (ms, clocks) of the
+    last region; clocks lists the rejected ones under "rejected_runs"."""
     multi = dist is not None and dist.is_initialized() and dist.get_world_size() > 1
     rejected = []
     for attempt in range(attempts):
@@ -301,9 +330,12 @@ def timed_replay(torch, graph, device, dist, sampler, attempts=2):
         torch.cuda.synchronize()
         with sampler() as clk:
             start.record()
-            graph.replay()
+            for _ in range(replays):
+                graph.replay()
             end.record()
             torch.cuda.synchronize()
+        if after is not None:
+            after()
         if multi:
             dist.barrier()
         ms, clocks = start.elapsed_time(end), clk.summary()
@@ -356,6 +388,32 @@ def step_batch(mxq, sets, k):
     return lambda: mxq.batch(ops)
 
 
+def decoder_stack(torch, seed=2):
+    """The 36 layers of seven bf16 [out, in] weights, N(0, 0.02), drawn on the device from a
+    seeded generator (the host generator's bits would take minutes at 3.6G values; parity on
+    those bits is a test)."""
+    dev = torch.device("cuda")
+    gen = torch.Generator(device=dev)
+    layers = []
+    for l in range(synthetic.N_LAYERS):
+        gen.manual_seed(seed * 1000 + l)
+        layers.append([(torch.randn(r, c, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+                       for _, r, c in synthetic.DECODER_LAYER])
+    return layers
+
+
+def stack_step(mxq, layers, outs):
+    """The 72 launches of one step: layer l to E2M3, then layer (l + 18) mod 36 to AXS-6, for
+    l = 0..35, so each launch reads a layer last read 18 layers earlier. outs[fmt][l] holds
+    layer l's preallocated codes and scales."""
+    L = len(layers)
+    fns = []
+    for l in range(L):
+        for fmt, j in ((STACK_FORMATS[0], l), (STACK_FORMATS[1], (l + L // 2) % L)):
+            fns.append(lambda ws=layers[j], o=outs[fmt][j], f=fmt: mxq.quantize_grouped(ws, f, outs=o))
+    return fns
+
+
 def graph_of(torch, fns):
     """One CUDA graph that launches every callable of `fns` in order on one stream."""
     g = torch.cuda.CUDAGraph()
@@ -396,26 +454,31 @@ def time_graph(torch, g, replays=1):
     return start.elapsed_time(end)
 
 
-def e2e_measure(torch, mxq, w_host, steps):
-    """Public API from pinned host memory, every step: H2D of the weight, one batch launch, D2H of
-    every output. The host->device copy of step k+1 runs on its own stream and overlaps the
-    device->host copies of step k (PCIe is full duplex); two device buffer sets alternate."""
+def e2e_measure(torch, mxq, steps):
+    """Public API from pinned host memory, one layer per step: the host->device copy of the
+    layer's seven weights, its grouped conversions to E2M3 and to AXS-6, the device->host copy
+    of both formats' codes and scales. The host->device copy of step k+1 runs on its own stream
+    and overlaps the device->host copies of step k (PCIe is full duplex); two device buffer sets
+    alternate, fed from two distinct pinned host layers."""
     dev = torch.device("cuda")
-    hx = torch.from_numpy(w_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+    gen = torch.Generator()
+    host = []
+    for h in range(2):
+        gen.manual_seed(2 * 1000 + h)
+        host.append([(torch.randn(r, c, generator=gen) * 0.02).to(torch.bfloat16).pin_memory()
+                     for _, r, c in synthetic.DECODER_LAYER])
     sets = []
     for _ in range(2):
-        x = torch.zeros_like(hx, device=dev)
-        ca, sa = mxq.quantize(x, "mxfp6_e2m3")
-        cb, sb = mxq.quantize(x, "mxfp6_e3m2")
-        sets.append({"x": x, "ca": ca, "sa": sa, "cb": cb, "sb": sb, "ya": torch.empty_like(x),
-                     "yb": torch.empty_like(x)})
-    outs_h = [torch.empty_like(sets[0][k], device="cpu").pin_memory() for k in ("ca", "sa", "cb", "sb", "ya", "yb")]
-    h2d = hx.numel() * 2
-    d2h = sum(o.numel() * o.element_size() for o in outs_h)
+        xs = [torch.empty_like(t, device=dev) for t in host[0]]
+        sets.append({"x": xs, "out": {f: mxq.quantize_grouped(xs, f) for f in STACK_FORMATS}})
+    outs_h = {f: [(torch.empty_like(c, device="cpu").pin_memory(), torch.empty_like(s, device="cpu").pin_memory())
+                  for c, s in sets[0]["out"][f]] for f in STACK_FORMATS}
+    h2d = sum(t.numel() * t.element_size() for t in host[0])
+    d2h = sum(c.numel() * c.element_size() + s.numel() * s.element_size() for f in STACK_FORMATS for c, s in outs_h[f])
     s_in, s_work = torch.cuda.Stream(), torch.cuda.Stream()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    done = [None, None]  # event after the batch that last read set p's input
+    done = [None, None]  # event after the conversions that last read set p's inputs
     torch.cuda.synchronize()
     for it in range(steps + 2):
         if it == 2:
@@ -423,29 +486,34 @@ def e2e_measure(torch, mxq, w_host, steps):
             s_work.synchronize()
             t0.record(s_in)
         p = it % 2
-        cur, prev = sets[p], sets[1 - p]
+        cur = sets[p]
         with torch.cuda.stream(s_in):
             if done[p] is not None:
                 s_in.wait_event(done[p])
-            cur["x"].copy_(hx, non_blocking=True)
+            for d, h in zip(cur["x"], host[it % 2]):
+                d.copy_(h, non_blocking=True)
             arrived = torch.cuda.Event()
             arrived.record(s_in)
         with torch.cuda.stream(s_work):
             s_work.wait_event(arrived)
-            mxq.batch([("quantize", "mxfp6_e2m3", cur["x"], cur["ca"], cur["sa"]),
-                       ("quantize", "mxfp6_e3m2", cur["x"], cur["cb"], cur["sb"]),
-                       ("dequantize", "mxfp6_e2m3", prev["ca"], prev["sa"], cur["ya"]),
-                       ("dequantize", "mxfp6_e3m2", prev["cb"], prev["sb"], cur["yb"])])
+            for f in STACK_FORMATS:
+                mxq.quantize_grouped(cur["x"], f, outs=cur["out"][f])
             done[p] = torch.cuda.Event()
             done[p].record(s_work)
-            for k, h in zip(("ca", "sa", "cb", "sb", "ya", "yb"), outs_h):
-                h.copy_(cur[k], non_blocking=True)
+            for f in STACK_FORMATS:
+                for (c, s), (hc, hs) in zip(cur["out"][f], outs_h[f]):
+                    hc.copy_(c, non_blocking=True)
+                    hs.copy_(s, non_blocking=True)
     t1.record(s_work)
     torch.cuda.synchronize()
+    mxq.check_device()
     ms = t0.elapsed_time(t1) / steps
-    step_bytes = 4 * nbytes_q("mxfp6_e2m3", hx.numel(), 2)
+    n = sum(t.numel() for t in host[0])
+    step_bytes = sum(nbytes_q(f, n, 2) for f in STACK_FORMATS)
     return {"value": round(step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms, 4),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "step": "one decoder layer: H2D of its 7 weights, grouped quantize to E2M3 and to AXS-6, D2H of both "
+                    "formats' codes and scales",
             "overlap": "H2D of step k+1 on its own stream during the D2H of step k"}
 
 
@@ -460,8 +528,8 @@ def time_launches(torch, fns, reps):
 
 
 def workloads_breakdown(torch, mxq, hbm):
-    """Device GB/s of every op of the five workloads (each launch reads HBM-resident
-    data: tensors above L2 size, or rotated copies; config 1 is latency-bound)."""
+    """Device GB/s of the ops of the other workloads (each launch reads HBM-resident data:
+    tensors above L2 size, or rotated copies; the 128x256 quick start is latency-bound)."""
     dev = torch.device("cuda")
     gen = torch.Generator(device=dev)
     out = {}
@@ -482,23 +550,38 @@ def workloads_breakdown(torch, mxq, hbm):
     rec("c1_axs6_quantize_f32", nbytes_q("axs6", n1, 4), n1, t[1])
     rec("c1_axs6_dequantize_f32", nbytes_q("axs6", n1, 4), n1, t[2])
 
-    # 3: the 36-layer decoder stack, one grouped launch per layer, MXFP6 E2M3 and AXS-6
-    shapes = synthetic.DECODER_LAYER
-    layers = []
-    for l in range(synthetic.N_LAYERS):
-        gen.manual_seed(2 * 1000 + l)
-        layers.append([(torch.randn(r, c, device=dev, generator=gen) * 0.02).to(torch.bfloat16) for _, r, c in shapes])
-    n3 = sum(r * c for _, r, c in shapes) * synthetic.N_LAYERS
-    for fmt in ("mxfp6_e2m3", "axs6"):
-        outs = [mxq.quantize_grouped(ws, fmt) for ws in layers]
-        fns = [lambda ws=ws, o=o: mxq.quantize_grouped(ws, fmt, outs=o) for ws, o in zip(layers, outs)]
-        g = graph_of(torch, fns * 2)
-        ms = time_graph(torch, g) / 2
+    # 2: the bf16 4096x4096 weight: one step = MXFP6 E2M3 + E3M2 quantize + dequantize in one batch
+    # launch, 8 rotating buffer sets (~1 GB: every launch reads data last touched >= 4 steps
+    # earlier); per_op: the four single-operation kernels, each a graph of 400 launches of it alone
+    w_host, _ = synthetic.weight_with_outliers(seed=1)
+    w = torch.from_numpy(w_host.view(np.int16)).view(torch.bfloat16).cuda()
+    sets = make_sets(torch, mxq, w, 8)
+    n2 = w.numel()
+    op_bytes = nbytes_q("mxfp6_e2m3", n2, 2)
+    K2 = 400
+    g = graph_of(torch, [step_batch(mxq, sets, k) for k in range(K2)])
+    upload_graph(torch, g)
+    ms = time_graph(torch, g) / K2
+    del g
+    rec("c2_weight_batch_step_bf16", 4 * op_bytes, 4 * n2, ms)
+    out["c2_weight_batch_step_bf16"]["launches"] = "one mxq_run_batch launch per step (the four conversions)"
+    for j, nm in enumerate([nm for nm, _ in step_ops(mxq, sets, 0)]):
+        g = graph_of(torch, [step_ops(mxq, sets, k)[j][1] for k in range(K2)])
+        ms = time_graph(torch, g) / K2
         del g
-        rec(f"c3_stack_{fmt}_quantize_bf16", nbytes_q(fmt, n3, 2), n3, ms)
-        del outs
-    del layers
+        rec(f"c2_weight_{nm}_bf16", op_bytes, n2, ms)
+    # column-direction blocks of the same weight (32 rows of a column), transposed layout: 8 launches
+    # per round on the 8 sets, so each reads data last touched 7 launches (330 MB) earlier
+    ccs = [mxq.quantize_cols(st["x"], "mxfp6_e2m3") for st in sets]
+    ts = time_launches(torch, [
+        lambda: [mxq.quantize_cols(st["x"], "mxfp6_e2m3", codes=c, scales=sc_) for st, (c, sc_) in zip(sets, ccs)],
+        lambda: [mxq.dequantize_cols(c, sc_, "mxfp6_e2m3", st["x"].shape, out=st["ya"])
+                 for st, (c, sc_) in zip(sets, ccs)]], 2)
+    rec("c2_weight_quantize_cols_e2m3_bf16", op_bytes, n2, ts[0] / len(sets))
+    rec("c2_weight_dequantize_cols_e2m3_bf16", op_bytes, n2, ts[1] / len(sets))
+    del sets, ccs, w
     torch.cuda.empty_cache()
+    mxq.check_device()
 
     # 4: activations bf16 16384x8192 (0.5*t3, 16 channels x100), gradients fp32 N(0,1e-3)
     gen.manual_seed(3)
@@ -519,7 +602,15 @@ def workloads_breakdown(torch, mxq, hbm):
         del c, s, y
     ts = time_launches(torch, [lambda: mxq.fake_quantize(g, "axs6", out=go)], 10)
     rec("c4_grad_axs6_fake_quantize_f32", 8 * g.numel(), g.numel(), ts[0])
-    del a, g, go
+    # column-direction blocks of the activations (the backward pass's K-contiguous operand)
+    cc, cs = mxq.quantize_cols(a, "mxfp6_e2m3")
+    y = torch.empty_like(a)
+    ts = time_launches(torch, [lambda: mxq.quantize_cols(a, "mxfp6_e2m3", codes=cc, scales=cs),
+                               lambda: mxq.dequantize_cols(cc, cs, "mxfp6_e2m3", a.shape, out=y)], 10)
+    rec("c4_act_quantize_cols_e2m3_bf16", nbytes_q("mxfp6_e2m3", a.numel(), 2), a.numel(), ts[0])
+    rec("c4_act_dequantize_cols_e2m3_bf16", nbytes_q("mxfp6_e2m3", a.numel(), 2), a.numel(), ts[1])
+    del a, g, go, cc, cs, y
+    mxq.check_device()
     torch.cuda.empty_cache()
 
     # 5: scores fp32 4096 x 32768 N(0,3) -> exp -> MXFP4
@@ -531,7 +622,13 @@ def workloads_breakdown(torch, mxq, hbm):
     rec("c5_scores_exp_mxfp4_f32", nbytes_q("mxfp4", sc.numel(), 4), sc.numel(), ts[0])
     # the same stage by the exp-free rule (no exponential), same bytes
     rec("c5_scores_exp_free_mxfp4_f32", nbytes_q("mxfp4", sc.numel(), 4), sc.numel(), ts[1])
+    for fmt in ("mxfp6_e2m3", "axs6"):
+        c6, s6 = mxq.exp_quantize(sc, fmt)
+        ts = time_launches(torch, [lambda: mxq.exp_quantize(sc, fmt, codes=c6, scales=s6)], 10)
+        rec(f"c5_scores_exp_{fmt}_f32", nbytes_q(fmt, sc.numel(), 4), sc.numel(), ts[0])
+        del c6, s6
     del sc, c5, s5
+    mxq.check_device()
     torch.cuda.empty_cache()
     return out
 
@@ -620,8 +717,8 @@ def main():
                     help="run one kernel a few times on its workload and exit (for ncu captures)")
     ap.add_argument("--profile-reps", type=int, default=3)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1600)
-    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="mxq", choices=["mxq", "reference"])
     ap.add_argument("--ref-seconds", type=float, default=20.0)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -647,84 +744,93 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
     hbm, how = peaks()
+    dd = dist if world > 1 else None
 
-    w_host, _ = synthetic.weight_with_outliers(seed=1)
-    w = torch.from_numpy(w_host.view(np.int16)).view(torch.bfloat16).cuda()
-    sets = make_sets(torch, mxq, w, 8)
-    n = w.numel()
-    op_bytes = nbytes_q("mxfp6_e2m3", n, 2)  # same for all four launches
-    step_bytes = 4 * op_bytes
+    # the stack (7.3 GB bf16) and both formats' outputs (5.8 GB), resident in HBM
+    layers = decoder_stack(torch)
+    outs = {f: [mxq.quantize_grouped(ws, f) for ws in layers] for f in STACK_FORMATS}
+    step = stack_step(mxq, layers, outs)
+    step_bytes, n = stack_step_bytes()
+    launches_per_step = len(step)
 
-    # warm-up: eager W steps, then the same W steps as a graph
-    for k in range(args.warmup):
-        step_batch(mxq, sets, k)()
+    # warm-up: W eager steps, then the step graph W times
+    for _ in range(args.warmup):
+        for fn in step:
+            fn()
     torch.cuda.synchronize()
-    names = [nm for nm, _ in step_ops(mxq, sets, 0)]
-    gw = graph_of(torch, [step_batch(mxq, sets, k) for k in range(args.warmup)])
-    gw.replay()
-    torch.cuda.synchronize()
-    # timed region: K steps (one batch launch of the four conversions each) as one graph
-    gt = graph_of(torch, [step_batch(mxq, sets, k) for k in range(args.warmup, args.warmup + args.steps)])
+    mxq.check_device()
+    gt = graph_of(torch, step)
     uploaded = upload_graph(torch, gt)
+    for _ in range(args.warmup):
+        gt.replay()
     torch.cuda.synchronize()
+    # timed region: the step graph replayed K times back to back
     uuid = getattr(torch.cuda.get_device_properties(local), "uuid", None)
-    ms_total, clocks = timed_replay(torch, gt, "cuda", dist if world > 1 else None,
-                                    lambda: ClockSampler(local, uuid=uuid))
-    del gt, gw
-    # the single-operation kernels, for comparison: K back-to-back launches of one (same rotation, cold data)
-    op_ms = {}
-    for j, nm in enumerate(names):
-        g = graph_of(torch, [step_ops(mxq, sets, k)[j][1] for k in range(args.steps)])
-        op_ms[nm] = time_graph(torch, g) / args.steps
+    ms_total, clocks = timed_replay(torch, gt, "cuda", dd, lambda: ClockSampler(local, uuid=uuid),
+                                    replays=args.steps, after=mxq.check_device)
+    del gt
+    ms_total = max_over_ranks(ms_total, dd, "cuda")
+    # each format's 36 launches alone, for the per-format figures (same layers, same rotation)
+    per_format = {}
+    for j, f in enumerate(STACK_FORMATS):
+        g = graph_of(torch, step[j::2])
+        ms = time_graph(torch, g, replays=max(3, min(args.steps, 10))) / max(3, min(args.steps, 10))
         del g
-    ms_total = max_over_ranks(ms_total, dist if world > 1 else None, "cuda")
+        b = nbytes_q(f, n, 2)
+        per_format[f] = {"ms_per_stack": round(ms, 4), "GB/s": round(b / (ms * 1e-3) / 1e9, 1),
+                         "Gelem/s": round(n / (ms * 1e-3) / 1e9, 1), "frac_hbm": round(b / (ms * 1e-3) / 1e9 / hbm, 4),
+                         "frac_nominal": round(b / (ms * 1e-3) / 1e9 / NOMINAL_HBM, 4), "bytes_per_stack": int(b)}
+    mxq.check_device()
+    del outs, layers, step
+    torch.cuda.empty_cache()
 
     ms_step = ms_total / args.steps
     value = job_gbs(world, step_bytes, args.steps, ms_total)
-    # the timed region launches one kernel only (the batch kernel, once per step): its average
-    # launch duration is the timed region's device time / K
-    ach = step_bytes / (ms_step * 1e-3) / 1e9
+    # the timed region launches the grouped quantize kernel only (its E2M3 and AXS-6 instances,
+    # 72 launches per step): algorithmic bytes per launch / average launch duration
+    bytes_per_launch = step_bytes / launches_per_step
+    ach = bytes_per_launch / (ms_step / launches_per_step * 1e-3) / 1e9
 
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "elements": n, "bytes_per_step": step_bytes,
+        "config": {"workload": WORKLOAD, "elements_per_step": 2 * n, "bytes_per_step": step_bytes,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "8 rotating buffer sets (~1 GB): each launch reads data last touched >= 4 steps earlier",
-                   "launches": "one mxq_run_batch launch per step (the four conversions)",
-                   "timing": "one CUDA graph of K steps replayed between CUDA events on the launching stream"
-                             + (", uploaded to the device before the timed replay" if uploaded else "")
-                             + "; per_op: the single-operation kernels, a graph of K launches of one alone"},
+                   "l2": "inputs larger than L2: each launch reads a 202 MB layer last read 18 layers "
+                         "(about 10 GB of traffic) earlier",
+                   "launches": f"{launches_per_step} mxq_quantize_grouped launches per step: layer l to E2M3, "
+                               "layer (l+18) mod 36 to AXS-6, l = 0..35",
+                   "timing": "one CUDA graph of one step replayed K times between CUDA events on the launching "
+                             "stream" + (", uploaded to the device first" if uploaded else "")
+                             + "; the device status word checked after the region"},
         "frac_hbm": round(value / world / hbm, 4),
-        "per_op": {nm: {"ms": round(v, 5), "GB/s": round(op_bytes / (v * 1e-3) / 1e9, 1),
-                        "Gelem/s": round(n / (v * 1e-3) / 1e9, 1),
-                        "frac_hbm": round(op_bytes / (v * 1e-3) / 1e9 / hbm, 4),
-                        "frac_nominal": round(op_bytes / (v * 1e-3) / 1e9 / NOMINAL_HBM, 4)}
-                   for nm, v in op_ms.items()},
-        "gelem_per_s": round(world * 4 * n * args.steps / (ms_total * 1e-3) / 1e9, 2),
-        "roofline": {"bound": "hbm", "kernel": "k_batch (4 conversions per launch)", "achieved": round(ach, 1),
-                     "peak": hbm, "peak_source": how, "unit": "GB/s", "frac": round(ach / hbm, 4),
-                     "peak_nominal": NOMINAL_HBM, "frac_nominal": round(ach / NOMINAL_HBM, 4),
-                     "traffic": ncu_traffic("batch_step"), "algorithmic_bytes_per_launch": step_bytes},
+        "per_format": per_format,
+        "gelem_per_s": round(world * 2 * n * args.steps / (ms_total * 1e-3) / 1e9, 2),
+        "roofline": {"bound": "hbm", "kernel": "grouped k_quantize<fmt, bf16, 64> (E2M3 and AXS-6 instances)",
+                     "achieved": round(ach, 1), "peak": hbm, "peak_source": how, "unit": "GB/s",
+                     "frac": round(ach / hbm, 4), "peak_nominal": NOMINAL_HBM,
+                     "frac_nominal": round(ach / NOMINAL_HBM, 4), "traffic": ncu_traffic("grouped_layer"),
+                     "algorithmic_bytes_per_launch": int(bytes_per_launch),
+                     "launch_ms": round(ms_step / launches_per_step, 5)},
         "clocks": clocks,
-        "gpu_launches": args.steps,
+        "gpu_launches": launches_per_step * args.steps,
     }
     if rank == 0:
-        result["e2e"] = e2e_measure(torch, mxq, w_host, steps=max(3, min(args.steps, 20)))
+        result["e2e"] = e2e_measure(torch, mxq, steps=max(3, min(args.steps, 12)))
         if not args.no_cpu_baseline:
-            v1, i1 = oracle_throughput(w_host, budget_s=args.cpu_seconds / 2)
+            pool = oracle_pool()
+            v1, i1 = oracle_throughput(pool, budget_s=args.cpu_seconds / 2)
             nt = cpu_threads()
-            vn, i_n = oracle_throughput(w_host, budget_s=args.cpu_seconds / 2, threads=nt)
+            vn, i_n = oracle_throughput(pool, budget_s=args.cpu_seconds / 2, threads=nt)
             result["cpu_baseline"] = {
                 "value": round(vn, 4), "unit": "GB/s", "cores": nt, "kind": "oracle",
-                "sample": f"{i_n['samples']} slices of 64 rows x 4096 (E2M3 and E3M2 quantize+dequantize), "
-                          f"{i_n['seconds']} s on {nt} threads",
+                "sample": f"{i_n['samples']} quantizations of 32-row slices of the stack's tensors (the workload's "
+                          f"own bits) to MXFP6 E2M3 and AXS-6, {i_n['elements']} values, {i_n['seconds']} s on "
+                          f"{nt} threads",
                 "single_thread": {"value": round(v1, 4), "cores": 1,
                                   "sample": f"{i1['samples']} slices, {i1['seconds']} s"}}
         if not args.no_workloads:
-            del sets
-            torch.cuda.empty_cache()
             result["workloads"] = workloads_breakdown(torch, mxq, hbm)
         print(json.dumps(result), flush=True)
     if world > 1:

@@ -7,9 +7,9 @@ CUDA kernels for NVIDIA B200 (sm_100a) behind a C ABI (include/mxq.h).
     w2 = dequantize(codes, scales, "mxfp6_e2m3", w_bf16.shape)
     g_q = fake_quantize(g_fp32, "axs6")          # quantize + dequantize, one pass
 """
-from .mxq import (EXPORTS, FORMATS, MXQError, batch, dequantize, dequantize_cols, dequantize_exmy, exp_quantize,
-                  fake_quantize, fake_quantize_exmy, lib, quantize, quantize_cols, quantize_exmy, quantize_grouped,
-                  quantize_mma, swizzle_scales)
+from .mxq import (EXPORTS, FORMATS, MXQError, batch, check_device, dequantize, dequantize_cols, dequantize_exmy,
+                  exp_free_quantize, exp_quantize, fake_quantize, fake_quantize_exmy, lib, quantize, quantize_cols,
+                  quantize_exmy, quantize_grouped, quantize_mma, swizzle_scales)
 
 
 def fake_quantize_ste(x, fmt="axs6", block_size=32):
@@ -18,6 +18,7 @@ def fake_quantize_ste(x, fmt="axs6", block_size=32):
     return f(x, fmt, block_size)
 
 
-__all__ = ["quantize", "dequantize", "fake_quantize", "fake_quantize_ste", "exp_quantize", "quantize_grouped",
+__all__ = ["quantize", "dequantize", "fake_quantize", "fake_quantize_ste", "exp_quantize", "exp_free_quantize",
+           "quantize_grouped", "check_device",
            "quantize_cols", "dequantize_cols", "quantize_exmy", "dequantize_exmy", "fake_quantize_exmy",
            "quantize_mma", "swizzle_scales", "batch", "MXQError", "FORMATS", "lib", "EXPORTS"]

@@ -293,8 +293,9 @@ mxq_status mxq_check_device(void) {
 
 mxq_status mxq_selftest_timeout(int limit_ms) {
     if (limit_ms < 1 || limit_ms > 1000) return MXQ_ERR_INVALID_ARG;
-    const mxq_status before = mxq_check_device();  // start from a clear word
-    if (before == MXQ_ERR_CUDA) return before;
+    // start from a clear word; a timeout left by an earlier call is reported, not cleared away
+    const mxq_status before = mxq_check_device();
+    if (before != MXQ_OK) return before;
     if (mxq::launch_selftest_timeout((unsigned long long)limit_ms * 1000000ull, 0) != cudaSuccess) return MXQ_ERR_CUDA;
     return mxq_check_device();
 }

@@ -462,7 +462,8 @@ static cudaError_t launch_qc_t(const void* src, void* codes, void* scales, long 
                                cudaStream_t st) {
     constexpr int TC = ColTile<T>::TC;
     CUtensorMap map;
-    if (encode_tile_map(&map, src, rows, cols, (int)sizeof(T))) {
+    // the tensor copy takes 32-bit coordinates: wider matrices take the one-shot kernel
+    if (cols <= 0x7FFFFFFFLL && rows <= 0x7FFFFFFFLL && encode_tile_map(&map, src, rows, cols, (int)sizeof(T))) {
         auto kern = k_quantize_cols_tma<F, T>;
         constexpr int smem = QColsSmem<F, T>::bytes;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -60,7 +60,7 @@ cudaError_t launch_fake_quantize_stream(int fmt, const void* src, void* dst, int
 cudaError_t launch_exp_quantize(int fmt, const float* scores, long long rows, long long cols, void* codes,
                                 void* scales, cudaStream_t st);
 bool exp_quantize_supported(long long cols);
-// bulk-copy pipeline form of the softmax stage (E2M1 and E4M3, scores 16-byte aligned)
+// bulk-copy pipeline form of the softmax stage (every format; scores 16-byte aligned)
 bool exp_quantize_tma_supported(int fmt, const void* scores);
 cudaError_t launch_exp_free_quantize(const float* scores, long long rows, long long cols, void* codes, void* scales,
                                      cudaStream_t st);

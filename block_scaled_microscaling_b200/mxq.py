@@ -245,6 +245,15 @@ def _check(status, what):
         raise MXQError(status, what)
 
 
+def _finish(check):
+    """check=True: synchronize and raise MXQError(MXQ_ERR_TIMEOUT) if a bounded wait of a kernel
+    ran out (its outputs are then incomplete). The bulk-copy kernels (exp_quantize,
+    exp_free_quantize, quantize_cols, fake_quantize of 2^19 blocks or more) bound their waits;
+    without check=True a caller learns of such a timeout only from a later check_device()."""
+    if check:
+        check_device()
+
+
 def _on_gpu(t, what):
     """The library computes on the GPU only: a host tensor is refused here, before any call."""
     if not t.is_cuda:
@@ -327,8 +336,10 @@ def _same_values(x, out):
     _fits(out, 0, "out")
 
 
-def fake_quantize(x, fmt="axs6", block_size=32, out=None, stream=None):
-    """Quantize then dequantize in one pass; out=x runs in place."""
+def fake_quantize(x, fmt="axs6", block_size=32, out=None, stream=None, check=False):
+    """Quantize then dequantize in one pass; out=x runs in place. Tensors of 2^19 blocks or more
+    go through a bulk-copy kernel with bounded waits: check=True synchronizes and raises if one
+    ran out (else call check_device() before trusting `out`)."""
     if block_size != 32:
         raise MXQError(4, f"block_size={block_size}")
     torch = _torch()
@@ -341,11 +352,14 @@ def fake_quantize(x, fmt="axs6", block_size=32, out=None, stream=None):
     rows, cols = _as2d(x)
     _check(mxq_fake_quantize(_fmt(fmt), x.data_ptr(), _dt(x), rows, cols, out.data_ptr(), _stream(stream)),
            "mxq_fake_quantize")
+    _finish(check)
     return out
 
 
-def exp_quantize(scores, fmt="mxfp4", codes=None, scales=None, stream=None):
-    """fp32 scores [..., keys] -> codes + scales of exp(s - rowmax), block-quantized per 32 keys."""
+def exp_quantize(scores, fmt="mxfp4", codes=None, scales=None, stream=None, check=False):
+    """fp32 scores [..., keys] -> codes + scales of exp(s - rowmax), block-quantized per 32 keys.
+    The kernel's waits are bounded: check=True synchronizes and raises if one ran out (else
+    call check_device() before trusting the outputs)."""
     torch = _torch()
     if scores.dtype != torch.float32 or not scores.is_contiguous():
         raise ValueError("scores must be contiguous float32")
@@ -360,12 +374,15 @@ def exp_quantize(scores, fmt="mxfp4", codes=None, scales=None, stream=None):
     _fits(scales, ns, "scales")
     _check(mxq_exp_quantize(_fmt(fmt), scores.data_ptr(), rows, cols, codes.data_ptr(), scales.data_ptr(),
                             _stream(stream)), "mxq_exp_quantize")
+    _finish(check)
     return codes, scales
 
 
-def exp_free_quantize(scores, codes=None, scales=None, stream=None):
+def exp_free_quantize(scores, codes=None, scales=None, stream=None, check=False):
     """fp32 scores [..., keys] -> MXFP4 codes + E8M0 scales by the exp-free rule (no exponential):
-    per 32 keys an exponent-only scale from the block's maximum, one affine map to E2M1 codes."""
+    per 32 keys an exponent-only scale from the block's maximum, one affine map to E2M1 codes.
+    The kernel's waits are bounded: check=True synchronizes and raises if one ran out (else
+    call check_device() before trusting the outputs)."""
     torch = _torch()
     if scores.dtype != torch.float32 or not scores.is_contiguous():
         raise ValueError("scores must be contiguous float32")
@@ -380,6 +397,7 @@ def exp_free_quantize(scores, codes=None, scales=None, stream=None):
     _fits(scales, ns, "scales")
     _check(mxq_exp_free_quantize(scores.data_ptr(), rows, cols, codes.data_ptr(), scales.data_ptr(), _stream(stream)),
            "mxq_exp_free_quantize")
+    _finish(check)
     return codes, scales
 
 
@@ -488,9 +506,11 @@ def quantize_grouped(xs, fmt, outs=None, stream=None):
     return outs
 
 
-def quantize_cols(x, fmt, codes=None, scales=None, stream=None):
+def quantize_cols(x, fmt, codes=None, scales=None, stream=None, check=False):
     """x [rows, cols] -> blocks of 32 rows per column, laid out as quantize(x.T):
-    codes [cols, rows/32*P], scales [cols, rows/32]."""
+    codes [cols, rows/32*P], scales [cols, rows/32]. The kernel's waits are bounded:
+    check=True synchronizes and raises if one ran out (else call check_device() before
+    trusting the outputs)."""
     if not x.is_contiguous() or x.dim() != 2:
         raise ValueError("x must be a contiguous 2-D tensor")
     _on_gpu(x, "x")
@@ -504,6 +524,7 @@ def quantize_cols(x, fmt, codes=None, scales=None, stream=None):
     _fits(scales, ns, "scales")
     _check(mxq_quantize_cols(_fmt(fmt), x.data_ptr(), _dt(x), rows, cols, codes.data_ptr(), scales.data_ptr(),
                              _stream(stream)), "mxq_quantize_cols")
+    _finish(check)
     return codes, scales
 
 

@@ -297,18 +297,26 @@ MXQ_API mxq_status mxq_swizzle_scales(const void* scales, int64_t rows, int64_t 
  * mxq_exp_free_quantize (every format and size), mxq_quantize_cols, and
  * mxq_fake_quantize on tensors of 2^19 blocks or more. Every such wait is
  * bounded (one second). A wait that runs out makes the kernel stop early,
- * leaving its outputs incomplete, and sets a device error word. mxq_check_device
- * synchronizes the current device and returns MXQ_ERR_TIMEOUT if that
- * happened since the last call (clearing the word), MXQ_ERR_CUDA if the device
- * reported an error, MXQ_OK otherwise. It is host-blocking; call it where a
- * synchronization is acceptable (after a step, in tests).
+ * leaving its outputs incomplete, and sets a device error word. The outputs of
+ * any call of these entry points are therefore undefined until a later
+ * mxq_check_device returns MXQ_OK: the call itself returns MXQ_OK when its
+ * launch succeeded, before the kernel has run. mxq_check_device synchronizes
+ * the current device and returns MXQ_ERR_TIMEOUT if a wait ran out since the
+ * last call (clearing the word), MXQ_ERR_CUDA if the device reported an error,
+ * MXQ_OK otherwise. It is host-blocking; call it where a synchronization is
+ * acceptable (after a step, in tests). There is one word per device, shared by
+ * every stream and host thread using that device: a check by one thread
+ * reports (and clears) a timeout of a kernel another thread launched.
  */
 MXQ_API mxq_status mxq_check_device(void);
-/* Self-test of that mechanism: launches one warp that waits on an mbarrier
- * nothing arrives at, with a limit of limit_ms milliseconds (1..1000), then
- * returns mxq_check_device(): MXQ_ERR_TIMEOUT when the wait gave up and was
- * reported as it should. Synchronizes the device. MXQ_ERR_INVALID_ARG for a
- * limit out of range. No counterpart on the pages: a diagnostic of the library. */
+/* Self-test of that mechanism: first runs mxq_check_device() and returns its
+ * status, without testing, if it is not MXQ_OK (a pending timeout of an
+ * earlier call is reported, not cleared away); then launches one warp that
+ * waits on an mbarrier nothing arrives at, with a limit of limit_ms
+ * milliseconds (1..1000), and returns mxq_check_device(): MXQ_ERR_TIMEOUT when
+ * the wait gave up and was reported as it should. Synchronizes the device.
+ * MXQ_ERR_INVALID_ARG for a limit out of range. No counterpart on the pages: a
+ * diagnostic of the library. */
 MXQ_API mxq_status mxq_selftest_timeout(int limit_ms);
 
 /* Bytes of the packed code array: rows * cols/32 * payload (0 on bad input). */

@@ -212,13 +212,39 @@ def test_ranks_agree_on_a_retake_gloo():
 
 
 def test_oracle_baseline_on_several_threads():
-    """The CPU baseline runs the oracle on independent row samples in several host threads at
-    once; each thread's samples are its own and the bytes add up over all of them."""
+    """The CPU baseline runs the oracle on independent row slices in several host threads at
+    once; each thread's slices are its own and the bytes add up over all of them."""
     import numpy as np
-    w = np.zeros((256, 4096), dtype=np.uint16)  # bf16 bits, four 64-row slices
-    v1, i1 = bench.oracle_throughput(w, budget_s=0.05)
-    v2, i2 = bench.oracle_throughput(w, budget_s=0.05, threads=2)
+    pool = [np.zeros((32, 2560), dtype=np.uint16), np.zeros((32, 9728), dtype=np.uint16)]  # bf16 bits
+    v1, i1 = bench.oracle_throughput(pool, budget_s=0.05)
+    v2, i2 = bench.oracle_throughput(pool, budget_s=0.05, threads=2)
     assert i1["threads"] == 1 and i2["threads"] == 2
     assert v1 > 0 and v2 > 0 and i2["samples"] >= 2
-    assert i2["elements"] == i2["samples"] * 64 * 4096
+    assert i1["elements"] == sum(pool[k % 2].size for k in range(i1["samples"]))
     assert 1 <= bench.cpu_threads() <= 32
+
+
+def test_oracle_pool_holds_the_workload_bits():
+    """The baseline's slices are rows of the decoder stack exactly as the generator draws them."""
+    import numpy as np
+    import synthetic
+    pool = bench.oracle_pool(n_slices=2, rows=2)
+    cols = {c for _, _, c in synthetic.DECODER_LAYER}
+    for xs in pool:
+        assert xs.dtype == np.uint16 and xs.shape[0] == 2 and xs.shape[1] in cols
+    # the first slice against the full tensor it was cut from
+    rng = np.random.default_rng(12345)
+    layer = int(rng.integers(synthetic.N_LAYERS))
+    k = int(rng.integers(len(synthetic.DECODER_LAYER)))
+    _, nrows, cols = synthetic.DECODER_LAYER[k]
+    r0 = int(rng.integers(nrows - 2 + 1))
+    w = synthetic.decoder_weight(layer, k)
+    assert np.array_equal(pool[0], w[r0:r0 + 2])
+
+
+def test_stack_step_bytes_are_the_survey_figures():
+    """Per layer 280 698 880 B to MXFP6 E2M3 and 283 852 800 B to AXS-6 (values in + codes +
+    scales), 36 layers per step."""
+    b, n = bench.stack_step_bytes()
+    assert n == 36 * 100925440
+    assert b == 36 * (280698880 + 283852800)

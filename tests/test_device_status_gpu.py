@@ -33,3 +33,16 @@ def test_pipeline_full_size_reports_ok():
     for fmt in ("mxfp4", "mxfp8"):
         mxq.exp_quantize(s, fmt)
     assert mxq.mxq_check_device() == 0
+
+
+def test_helpers_check_on_request():
+    """check=True on the bulk-copy helpers synchronizes and reads the status word: a clean run
+    returns normally (a timed-out one would raise MXQError with MXQ_ERR_TIMEOUT)."""
+    s = torch.randn(64, 4096, device="cuda") * 3
+    mxq.exp_quantize(s, "mxfp4", check=True)
+    mxq.exp_free_quantize(s, check=True)
+    x = torch.randn(512, 256, device="cuda")
+    mxq.quantize_cols(x, "mxfp6_e2m3", check=True)
+    g = torch.randn(1 << 19, 32, device="cuda")  # 2^19 blocks: the bulk-copy fake-quantize
+    mxq.fake_quantize(g, "axs6", check=True)
+    assert mxq.mxq_check_device() == 0
