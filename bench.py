@@ -635,7 +635,9 @@ def workloads_breakdown(torch, mxq, hbm):
 
 PROFILE_CASES = ["batch_weight", "q_e2m3_weight", "q_e3m2_weight", "dq_e2m3_weight", "q_mxfp8_act", "dq_mxfp8_act", "q_axs6_layer",
                  "q_e2m3_layer", "fq_axs6_grad", "exp_mxfp4_scores", "expfree_mxfp4_scores", "qcols_e2m3_weight",
-                 "dqcols_e2m3_weight", "exmy_e3m3_act", "dq_exmy_e3m3_act", "fq_exmy_e3m3_act", "qmma_mxfp8_act"]
+                 "dqcols_e2m3_weight", "qcols_e2m3_act", "dqcols_e2m3_act", "exmy_e3m3_act", "dq_exmy_e3m3_act",
+                 "fq_exmy_e3m3_act", "qmma_mxfp8_act", "dq_e2m3_act", "fq_axs6_quickstart",
+                 "swizzle_scales_act", "exp_e2m3_scores", "exp_axs6_scores"]
 
 
 def profile_case(name, reps):
@@ -664,6 +666,31 @@ def profile_case(name, reps):
             fn = lambda: mxq.quantize(x, f, codes=c, scales=s)
         else:
             fn = lambda: mxq.dequantize(c, s, f, x.shape, out=y)
+    elif name in ("qcols_e2m3_act", "dqcols_e2m3_act"):
+        x = (torch.randn(16384, 8192, device=dev, generator=gen) * 0.5).to(torch.bfloat16)
+        cc, cs = mxq.quantize_cols(x, "mxfp6_e2m3")
+        y = torch.empty_like(x)
+        fn = (lambda: mxq.quantize_cols(x, "mxfp6_e2m3", codes=cc, scales=cs)) if name[0] == "q" else \
+            (lambda: mxq.dequantize_cols(cc, cs, "mxfp6_e2m3", x.shape, out=y))
+    elif name == "dq_e2m3_act":
+        x = (torch.randn(16384, 8192, device=dev, generator=gen) * 0.5).to(torch.bfloat16)
+        c, s = mxq.quantize(x, "mxfp6_e2m3")
+        y = torch.empty_like(x)
+        fn = lambda: mxq.dequantize(c, s, "mxfp6_e2m3", x.shape, out=y)
+    elif name == "fq_axs6_quickstart":
+        x = torch.randn(128, 256, device=dev, generator=gen)
+        o = torch.empty_like(x)
+        fn = lambda: mxq.fake_quantize(x, "axs6", out=o)
+    elif name == "swizzle_scales_act":
+        x = (torch.randn(16384, 8192, device=dev, generator=gen) * 0.5).to(torch.bfloat16)
+        _, s = mxq.quantize(x, "mxfp8")
+        o = mxq.swizzle_scales(s)
+        fn = lambda: mxq.swizzle_scales(s, out=o)
+    elif name in ("exp_e2m3_scores", "exp_axs6_scores"):
+        fmt = "mxfp6_e2m3" if "e2m3" in name else "axs6"
+        sc = torch.randn(4096, 32768, device=dev, generator=gen) * 3
+        c, s = mxq.exp_quantize(sc, fmt)
+        fn = lambda: mxq.exp_quantize(sc, fmt, codes=c, scales=s)
     elif name in ("exmy_e3m3_act", "dq_exmy_e3m3_act", "fq_exmy_e3m3_act"):
         x = (torch.randn(16384, 8192, device=dev, generator=gen) * 0.5).to(torch.bfloat16)
         c, s = mxq.quantize_exmy(x, 3, 3)

@@ -457,6 +457,292 @@ __global__ void __launch_bounds__(kColThreads) k_dequantize_cols(const void* __r
     }
 }
 
+// the 16 codes k = 16h .. 16h+15 of a payload start at word h * W / 2 (W-bit codes, 16 per
+// half): hw gets that half's W/2 words
+template <int F>
+__device__ __forceinline__ void load_half_payload(const uint8_t* block, int h, uint32_t* hw) {
+    constexpr int NH = Fmt<F>::W / 2;
+    const uint32_t* q = reinterpret_cast<const uint32_t*>(block) + h * NH;
+#pragma unroll
+    for (int i = 0; i < NH; ++i) hw[i] = q[i];
+}
+
+// true when a half payload holds an E4M3 NaN magnitude (0x7F)
+template <int F> __device__ __forceinline__ bool half_has_nan(const uint32_t* hw) {
+    if constexpr (F == F_E4M3) {
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m |= ((hw[i] & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u;
+        return m != 0;
+    } else {
+        return false;
+    }
+}
+
+// ---- dequantize to bf16: persistent, payloads prefetched two tiles ahead --------------------------
+//
+// Tiles of 256 rows x 64 columns (128-byte output rows, one whole line per row; a column's 8
+// row-blocks of payload are one 192-byte run on a 64-byte boundary: whole DRAM accesses). Each
+// CTA walks tiles blockIdx.x + n * gridDim.x in band-major order (the CTAs running at one time
+// cover a few adjacent row bands, so the rows they write are close together) and keeps the loads
+// of tiles n + 1 and n + 2 in flight while it decodes and stores tile n: the payloads come in by
+// 8-byte cp.async copies into a ring of three stages, the scales by plain loads into a register
+// that is written to its stage one iteration later. cp.async waits are the hardware's own (no
+// spin on a flag), so no wait here needs a bound.
+// Decode: warp w takes row-blocks (w & 3) and (w & 3) + 4 of column group w >> 2 (32 columns);
+// lane L columns 2p, 2p + 1 of the group (p = L & 15), rows 16h .. 16h + 15 of each row-block
+// (h = L >> 4), so each decoded word is one row's pair of neighbouring columns.
+constexpr int kDqCols = 64, kDqRbt = 8, kDqRows = 32 * kDqRbt, kDqStages = 3;
+
+template <int F> struct DqStage {
+    static constexpr int PB = payload<F>(), SB = Fmt<F>::FIXED ? 2 : 1;
+    static constexpr int CS = kDqRbt * PB + 8;                      // padded column stride of the payloads
+    static constexpr int SC = kDqCols * CS;                          // offset of the scales
+    static constexpr int bytes = (SC + kDqCols * kDqRbt * SB + 15) / 16 * 16;
+};
+
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// chunk swizzle of output row r (16-byte chunk c stored at c ^ dq_swz(r)): bits 0 and 2 from
+// r & 3 spread out, bit 2 flipped by r & 16. The decoding lanes of one row index write rows 16
+// apart (bit 4 of r) into different banks; the 4 rows x 2 threads of a quarter-warp reading
+// chunks {2hf + c} of their rows cover all banks.
+__device__ __forceinline__ int dq_swz(int r) { return ((r & 1) | ((r & 2) << 1)) ^ (((r >> 4) & 1) << 2); }
+
+// tile coordinates of tiles first, first + step, ... (band-major: tx fastest), by additions
+struct DqWalk {
+    int tx, by, ntx, nby, dx, dy;
+    __device__ __forceinline__ DqWalk(int ntx_, int nby_) : ntx(ntx_), nby(nby_) {
+        const int G = (int)gridDim.x, b = (int)blockIdx.x;
+        tx = b % ntx;
+        by = b / ntx;
+        dx = G % ntx;
+        dy = G / ntx;
+    }
+    __device__ __forceinline__ bool valid() const { return by < nby; }
+    __device__ __forceinline__ void next() {
+        tx += dx;
+        by += dy;
+        if (tx >= ntx) {
+            tx -= ntx;
+            ++by;
+        }
+    }
+};
+
+// 16 values of a column (rows 16h .. 16h + 15 of a row-block) as exact f32 values: the
+// up-conversions for the floating-point formats; AXS-6 by placing its magnitude on the fp32 fields
+// (cheaper there than converting m to float, by measurement)
+template <int F> __device__ __forceinline__ void dq_vals16(const uint32_t* hw, float* v) {
+    if constexpr (F == F_AXS6) {
+        const unsigned long long D = dup2(decode_unit<F>());
+#pragma unroll
+        for (int k = 0; k < 16; k += 2)
+            upk(f2mul(pk(__uint_as_float(payload_bits<F>(hw, k)), __uint_as_float(payload_bits<F>(hw, k + 1))), D), v[k],
+                v[k + 1]);
+    } else {
+        decode16<F>(hw, v);
+    }
+}
+
+// Sizes: every byte offset into the codes, scales and output fits in 31 bits (the launcher
+// checks), so the per-tile arithmetic is 32-bit.
+template <int F>
+__global__ void __launch_bounds__(kColThreads, 2) k_dequantize_cols_bf16(const void* __restrict__ codes,
+                                                                        const void* __restrict__ scales,
+                                                                        void* __restrict__ dst, int rows, int cols) {
+    using St = DqStage<F>;
+    constexpr int PB = St::PB, SB = St::SB, CS = St::CS;
+    constexpr int SEG8 = kDqRbt * PB / 8;             // 8-byte pieces of one column's payloads in a tile
+    constexpr int NU = kDqCols * SEG8 / kColThreads;  // this thread's pieces of a full tile
+    static_assert(kDqCols * SEG8 % kColThreads == 0, "whole pieces per thread");
+    extern __shared__ __align__(16) uint8_t dsm[];
+    uint8_t* const tile = dsm;                    // kDqRows x 128 bytes
+    uint8_t* const stages = dsm + kDqRows * 128;  // kDqStages x St::bytes
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int RB = rows / 32;
+    const int nby = (rows + kDqRows - 1) / kDqRows;
+    const int ntx = (cols + kDqCols - 1) / kDqCols;
+    const bool a32 = ((reinterpret_cast<uintptr_t>(dst) | (uintptr_t)(cols * 2)) & 31) == 0;
+    const uint32_t st0 = smem_u32(stages);
+    const int col_bytes = RB * PB;  // one column's payloads in the transposed layout
+    // a column's scales of a full tile are one aligned 8-byte (AXS-6: 16-byte) load when the
+    // column's scale run starts on that boundary
+    const bool wide_scales = RB % kDqRbt == 0 && (reinterpret_cast<uintptr_t>(scales) & (kDqRbt * SB - 1)) == 0;
+    const char* const cbase = reinterpret_cast<const char*>(codes);
+    const char* const sbase = reinterpret_cast<const char*>(scales);
+    char* const dbase = reinterpret_cast<char*>(dst);
+
+    // per-thread offsets, the same for every full tile: its NU payload pieces (shared, and global
+    // relative to the tile's first column run) and its column's scale run
+    uint32_t so_u[NU];
+    int go_u[NU];
+#pragma unroll
+    for (int u = 0; u < NU; ++u) {
+        const int i = t + u * kColThreads, j = i / SEG8, k = i - j * SEG8;
+        so_u[u] = (uint32_t)(j * CS + 8 * k);
+        go_u[u] = j * col_bytes + 8 * k;
+    }
+    const int gs_t = t * RB * SB;  // column t's scale run (bytes), t < kDqCols
+
+    bool swide = false;  // the pending scale registers hold a whole column's run
+    uint4 sw = make_uint4(0, 0, 0, 0);
+    // copies of the tile at `w` into stage `stage` (one commit group per tile, empty past the last
+    // tile); this thread's scale(s) of the tile are loaded into registers, to be stored later
+    auto issue = [&](const DqWalk& w, int stage, int& soff) {
+        soff = -1;
+        swide = false;
+        if (w.valid()) {
+            const int col0 = w.tx * kDqCols;
+            const int ncols = min(kDqCols, cols - col0);
+            const int nrb = min(kDqRbt, RB - w.by * kDqRbt);
+            const int tb = col0 * RB + w.by * kDqRbt;  // first column's first row-block
+            const char* src = cbase + tb * PB;
+            const uint32_t sb = st0 + (uint32_t)(stage * St::bytes);
+            if (ncols == kDqCols && nrb == kDqRbt) {
+#pragma unroll
+                for (int u = 0; u < NU; ++u) cp_async8(sb + so_u[u], src + go_u[u]);
+            } else {
+                const int seg8 = nrb * PB / 8;
+                for (int i = t; i < ncols * seg8; i += kColThreads) {
+                    const int j = i / seg8, k = i % seg8;
+                    cp_async8(sb + (uint32_t)(j * CS + 8 * k), src + j * col_bytes + 8 * k);
+                }
+            }
+            if (wide_scales && nrb == kDqRbt) {  // a column's kDqRbt scales in one aligned load
+                if (t < ncols) {
+                    const char* g = sbase + tb * SB + gs_t;
+                    if constexpr (SB == 2) {
+                        sw = __ldg(reinterpret_cast<const uint4*>(g));
+                    } else {
+                        const uint2 v = __ldg(reinterpret_cast<const uint2*>(g));
+                        sw.x = v.x;
+                        sw.y = v.y;
+                    }
+                    soff = stage * St::bytes + St::SC + t * kDqRbt * SB;
+                    swide = true;
+                }
+            } else {
+                for (int i = t; i < ncols * nrb; i += kColThreads) {  // byte by byte, straight to the stage
+                    const int j = i / nrb, k = i - (i / nrb) * nrb;
+                    const int g = tb + j * RB + k;
+                    const int off = stage * St::bytes + St::SC + (j * kDqRbt + k) * SB;
+                    if constexpr (SB == 2) *reinterpret_cast<uint16_t*>(stages + off) = __ldg(reinterpret_cast<const uint16_t*>(scales) + g);
+                    else stages[off] = __ldg(reinterpret_cast<const uint8_t*>(scales) + g);
+                }
+            }
+        }
+        cp_async_commit();
+    };
+    auto put_scale = [&](int soff) {
+        if (soff < 0 || !swide) return;
+        if constexpr (SB == 2) *reinterpret_cast<uint4*>(stages + soff) = sw;
+        else *reinterpret_cast<uint2*>(stages + soff) = make_uint2(sw.x, sw.y);
+    };
+
+    // decode role: row-blocks rb and rb + 4 of column group cg; columns ja, ja + 1, rows 16h ..
+    const int rb = warp & 3, cg = warp >> 2;
+    const int p = lane & 15, h = lane >> 4;
+    const int ja = cg * 32 + 2 * p;
+    const int pa_off = ja * CS + rb * PB, sa_off = St::SC + (ja * kDqRbt + rb) * SB;
+    uint8_t* const obase = tile + (rb * 32 + 16 * h) * 128 + 4 * (p & 3);
+    uint32_t c16[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) c16[q] = (uint32_t)(16 * ((4 * cg + (p >> 2)) ^ dq_swz(q + 16 * h)));
+    // store role: thread (r, hf) stores bytes 32hf .. 32hf + 31 of output rows r and r + 128 and,
+    // in a full 64-column strip, bytes 64 + 32hf .. (a strip of 32 columns is 64 bytes)
+    const int r = t >> 1, hf = t & 1;
+    uint32_t rd[4];  // byte offsets of its four chunks of row r in the output tile (row r + 128: + 128 * 128)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) rd[c] = (uint32_t)(r * 128 + 16 * (((c & 1) + 2 * hf + 4 * (c >> 1)) ^ dq_swz(r)));
+    const int rowoff = r * cols * 2 + 32 * hf;
+
+    DqWalk cur(ntx, nby), ahead(ntx, nby);
+    int so = -1;
+    issue(ahead, 0, so);
+    put_scale(so);  // the first tile's scales: one exposed load latency per CTA
+    ahead.next();
+    issue(ahead, 1, so);
+    ahead.next();
+    for (int stage = 0; cur.valid(); cur.next(), stage = stage == kDqStages - 1 ? 0 : stage + 1) {
+        const int col0 = cur.tx * kDqCols, row0 = cur.by * kDqRows;
+        const int ncols = min(kDqCols, cols - col0);
+        const int nrows = min(kDqRows, rows - row0);
+        cp_async_wait<1>();  // this thread's copies of the tile have landed
+        __syncthreads();     // everyone's have; the previous tile's rows have left the output tile
+        const uint8_t* stg = stages + stage * St::bytes;
+        if (cg * 32 < ncols) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                if (rb + 4 * half >= nrows / 32) break;
+                const uint8_t* sp = stg + pa_off + half * 4 * PB;
+                uint32_t ha[Fmt<F>::W / 2], hb[Fmt<F>::W / 2];
+                load_half_payload<F>(sp, h, ha);
+                load_half_payload<F>(sp + CS, h, hb);
+                uint32_t ba, bb;
+                if constexpr (SB == 2) {
+                    ba = *reinterpret_cast<const uint16_t*>(stg + sa_off + half * 4 * SB) & 0xFFu;
+                    bb = *reinterpret_cast<const uint16_t*>(stg + sa_off + half * 4 * SB + kDqRbt * SB) & 0xFFu;
+                } else {
+                    ba = stg[sa_off + half * 4];
+                    bb = stg[sa_off + half * 4 + kDqRbt];
+                }
+                float va[16], vb[16];
+                dq_vals16<F>(ha, va);
+                dq_vals16<F>(hb, vb);
+                const unsigned long long S = pk(fwd_scale(ba), fwd_scale(bb));
+                uint32_t o[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    float x, y;
+                    upk(f2mul(pk(va[k], vb[k]), S), x, y);
+                    o[k] = bf16x2(x, y);
+                }
+                if (ba == 0xFFu || bb == 0xFFu || half_has_nan<F>(ha) || half_has_nan<F>(hb)) {
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {  // canonical quiet NaN for NaN blocks and E4M3 NaN codes
+                        const bool na = ba == 0xFFu || (F == F_E4M3 && ((ha[k >> 2] >> (8 * (k & 3))) & 0x7Fu) == 0x7Fu);
+                        const bool nb = bb == 0xFFu || (F == F_E4M3 && ((hb[k >> 2] >> (8 * (k & 3))) & 0x7Fu) == 0x7Fu);
+                        if (na) o[k] = (o[k] & 0xFFFF0000u) | 0x7FC0u;
+                        if (nb) o[k] = (o[k] & 0x0000FFFFu) | 0x7FC00000u;
+                    }
+                }
+                uint8_t* ob = obase + half * 128 * 128;  // row-block rb + 4: 128 rows further
+#pragma unroll
+                for (int k = 0; k < 16; ++k) *reinterpret_cast<uint32_t*>(ob + k * 128 + c16[k & 3]) = o[k];
+            }
+        }
+        __syncthreads();  // the output tile is complete; this stage is free
+        put_scale(so);    // the next tile's scales into its stage (read after the next barrier)
+        issue(ahead, stage == 0 ? kDqStages - 1 : stage - 1, so);
+        ahead.next();
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            if (r + 128 * half < nrows) {
+                char* q = dbase + ((row0 + 128 * half) * cols + col0) * 2 + rowoff;
+                uint32_t w[16];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(tile + rd[c] + half * 128 * 128);
+                    w[4 * c] = v.x;
+                    w[4 * c + 1] = v.y;
+                    w[4 * c + 2] = v.z;
+                    w[4 * c + 3] = v.w;
+                }
+                st32(q, w, a32);
+                if (ncols == kDqCols) st32(q + 64, w + 8, a32);
+            }
+        }
+    }
+    cp_async_wait<0>();  // no copy may land in shared memory after the CTA has left
+}
+
+template <int F> static constexpr int dq_bf16_smem() { return kDqRows * 128 + kDqStages * DqStage<F>::bytes; }
+
 template <int F, typename T>
 static cudaError_t launch_qc_t(const void* src, void* codes, void* scales, long long rows, long long cols,
                                cudaStream_t st) {
@@ -487,6 +773,29 @@ static cudaError_t launch_qc_t(const void* src, void* codes, void* scales, long 
 template <int F, typename T>
 static cudaError_t launch_dqc_t(const void* codes, const void* scales, void* dst, long long rows, long long cols,
                                 cudaStream_t st) {
+    if constexpr (sizeof(T) == 2) {
+        // 32-bit offsets: the outputs, the codes and the scales each below 2^31 bytes
+        if (rows * cols * 2 < (1LL << 31) && rows * (cols / 32) * payload<F>() < (1LL << 31)) {
+            auto kern = k_dequantize_cols_bf16<F>;
+            constexpr int smem = dq_bf16_smem<F>();
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) return e;
+            int dev = 0, sms = 148, per_sm = 1;
+            cudaGetDevice(&dev);
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kColThreads, smem);
+            // two CTAs per SM, though shared memory would hold three: the 8-byte copies are staged
+            // through L1, and a third CTA's stages leave L1 too small for them (bf16 16384x8192,
+            // fraction of the HBM peak, E2M3 / E4M3 / E2M1: 0.57 / 0.90 / 0.80 with three CTAs,
+            // 0.81 / 0.92 / 0.84 with two)
+            if (per_sm > 2) per_sm = 2;
+            const long long ntiles = ((cols + kDqCols - 1) / kDqCols) * ((rows + kDqRows - 1) / kDqRows);
+            long long grid = (long long)sms * (per_sm > 0 ? per_sm : 1);
+            if (grid > ntiles) grid = ntiles;
+            kern<<<(unsigned)grid, kColThreads, smem, st>>>(codes, scales, dst, (int)rows, (int)cols);
+            return cudaGetLastError();
+        }
+    }
     dim3 grid((unsigned)(cols / kNarrowCols), (unsigned)((rows + kTileRows - 1) / kTileRows));
     k_dequantize_cols<F, T><<<grid, kColThreads, 0, st>>>(codes, scales, dst, rows, cols);
     return cudaGetLastError();

@@ -10,8 +10,10 @@
 // Rounding uses the sm_100a conversion instructions
 // cvt.rn.satfinite.{e2m3x2,e3m2x2,e4m3x2,e2m1x2}.f32 (round to nearest even,
 // saturate to the largest finite value), two values per instruction; AXS-6
-// rounds with a float add of 1.5*2^23. Decoding places the magnitude bits
-// into an fp32 bit pattern and rescales by exact powers of two.
+// rounds with a float add of 1.5*2^23. Decoding either places the magnitude
+// bits into an fp32 bit pattern and rescales by exact powers of two, or (the
+// column-direction dequantize) takes the exact values from the up-conversions
+// cvt.rn.f16x2.{e2m3x2,e3m2x2,e4m3x2,e2m1x2} and multiplies by the scale.
 #pragma once
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -307,6 +309,89 @@ __device__ __forceinline__ void decode2(uint32_t c0, uint32_t c1, float s, float
     v1 = __uint_as_float(code_to_bits<F>(c1));
     mul2(v0, v1, decode_unit<F>());
     mul2(v0, v1, s);
+}
+
+// ---------------------------------------------------------------------------
+// exact element values by the sm_100a up-conversions: cvt.rn.f16x2.{e2m3x2,e3m2x2,e4m3x2} turns
+// two codes (one per byte of a 16-bit operand, low byte -> low half) into their f16 values,
+// cvt.rn.f16x2.e2m1x2 two nibbles of a byte. Every value of these formats is an f16 normal or
+// zero, so the conversion is exact (an E4M3 NaN code gives an f16 NaN); the f16 -> f32 widening
+// is exact too.
+
+// four codes, one per byte of x (6-bit codes in the low 6 bits, 8-bit codes whole) -> f32 values
+template <int F>
+__device__ __forceinline__ void up4(uint32_t x, float& v0, float& v1, float& v2, float& v3) {
+    static_assert(F == F_E2M3 || F == F_E3M2 || F == F_E4M3, "byte-wide codes");
+    if constexpr (F == F_E2M3)
+        asm("{ .reg .b16 lo, hi; .reg .b32 a, b; .reg .f16 a0, a1, b0, b1;\n"
+            "mov.b32 {lo, hi}, %4;\n"
+            "cvt.rn.f16x2.e2m3x2 a, lo;\n cvt.rn.f16x2.e2m3x2 b, hi;\n"
+            "mov.b32 {a0, a1}, a;\n mov.b32 {b0, b1}, b;\n"
+            "cvt.f32.f16 %0, a0;\n cvt.f32.f16 %1, a1;\n cvt.f32.f16 %2, b0;\n cvt.f32.f16 %3, b1; }"
+            : "=f"(v0), "=f"(v1), "=f"(v2), "=f"(v3) : "r"(x));
+    else if constexpr (F == F_E3M2)
+        asm("{ .reg .b16 lo, hi; .reg .b32 a, b; .reg .f16 a0, a1, b0, b1;\n"
+            "mov.b32 {lo, hi}, %4;\n"
+            "cvt.rn.f16x2.e3m2x2 a, lo;\n cvt.rn.f16x2.e3m2x2 b, hi;\n"
+            "mov.b32 {a0, a1}, a;\n mov.b32 {b0, b1}, b;\n"
+            "cvt.f32.f16 %0, a0;\n cvt.f32.f16 %1, a1;\n cvt.f32.f16 %2, b0;\n cvt.f32.f16 %3, b1; }"
+            : "=f"(v0), "=f"(v1), "=f"(v2), "=f"(v3) : "r"(x));
+    else
+        asm("{ .reg .b16 lo, hi; .reg .b32 a, b; .reg .f16 a0, a1, b0, b1;\n"
+            "mov.b32 {lo, hi}, %4;\n"
+            "cvt.rn.f16x2.e4m3x2 a, lo;\n cvt.rn.f16x2.e4m3x2 b, hi;\n"
+            "mov.b32 {a0, a1}, a;\n mov.b32 {b0, b1}, b;\n"
+            "cvt.f32.f16 %0, a0;\n cvt.f32.f16 %1, a1;\n cvt.f32.f16 %2, b0;\n cvt.f32.f16 %3, b1; }"
+            : "=f"(v0), "=f"(v1), "=f"(v2), "=f"(v3) : "r"(x));
+}
+// eight E2M1 codes, one per nibble of x (code k in nibble k) -> f32 values
+__device__ __forceinline__ void up8_e2m1(uint32_t x, float* v) {
+    asm("{ .reg .b8 c0, c1, c2, c3; .reg .b32 a, b, c, d; .reg .f16 a0, a1, b0, b1, e0, e1, d0, d1;\n"
+        "mov.b32 {c0, c1, c2, c3}, %8;\n"
+        "cvt.rn.f16x2.e2m1x2 a, c0;\n cvt.rn.f16x2.e2m1x2 b, c1;\n"
+        "cvt.rn.f16x2.e2m1x2 c, c2;\n cvt.rn.f16x2.e2m1x2 d, c3;\n"
+        "mov.b32 {a0, a1}, a;\n mov.b32 {b0, b1}, b;\n mov.b32 {e0, e1}, c;\n mov.b32 {d0, d1}, d;\n"
+        "cvt.f32.f16 %0, a0;\n cvt.f32.f16 %1, a1;\n cvt.f32.f16 %2, b0;\n cvt.f32.f16 %3, b1;\n"
+        "cvt.f32.f16 %4, e0;\n cvt.f32.f16 %5, e1;\n cvt.f32.f16 %6, d0;\n cvt.f32.f16 %7, d1; }"
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+        : "r"(x));
+}
+
+// Sixteen consecutive codes of a payload, starting at a word boundary (hw: their W/2 words), as
+// exact f32 values of the element format (AXS-6: m/16 with the sign; E4M3 NaN codes: NaN).
+// 6-bit codes are spread to one per byte first: a 24-bit group c0 | c1 << 6 | c2 << 12 | c3 << 18
+// becomes c0 | c1 << 8 | c2 << 16 | c3 << 24 in two shift-and-merge steps.
+template <int F>
+__device__ __forceinline__ void decode16(const uint32_t* hw, float* v) {
+    if constexpr (F == F_E4M3) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) up4<F>(hw[i], v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    } else if constexpr (F == F_E2M1) {
+        up8_e2m1(hw[0], v);
+        up8_e2m1(hw[1], v + 8);
+    } else {
+        uint32_t g[4];
+        g[0] = hw[0];
+        g[1] = __funnelshift_r(hw[0], hw[1], 24);
+        g[2] = __funnelshift_r(hw[1], hw[2], 16);
+        g[3] = hw[2] >> 8;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            // bits 24.. of a group are the next group's: the masks below drop them
+            const uint32_t y = (g[i] & 0x0000FFFFu) | ((g[i] << 4) & 0xFFFF0000u);
+            const uint32_t z = ((y & 0x003F003Fu) | ((y << 2) & 0x3F003F00u));
+            if constexpr (F == F_AXS6) {
+                // sign | 5-bit magnitude m, value m / 16: the magnitude converted exactly, the sign copied
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t c = z >> (8 * k);
+                    v[4 * i + k] = __uint_as_float(__float_as_uint((float)(c & 31u) * 0.0625f) | ((c & 32u) << 26));
+                }
+            } else {
+                up4<F>(z, v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
+        }
+    }
 }
 
 // fp32 pair -> bf16x2, round to nearest even
