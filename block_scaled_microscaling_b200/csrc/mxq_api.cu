@@ -165,7 +165,8 @@ mxq_status mxq_quantize_mma(mxq_format fmt, const void* src, mxq_dtype dtype, in
 }
 
 mxq_status mxq_swizzle_scales(const void* scales, int64_t rows, int64_t kblocks, void* out, mxq_stream stream) {
-    if (rows < 0 || kblocks <= 0 || kblocks > kMaxElems / 32) return MXQ_ERR_SHAPE;
+    // a tile-row's 4-byte output words are counted in 32 bits: kblocks up to 4 * (2^31 - 1) / 128
+    if (rows < 0 || kblocks <= 0 || kblocks > kMaxElems / 32 || kblocks > 4 * (0x7FFFFFFFLL / 128)) return MXQ_ERR_SHAPE;
     MXQ_TRY(check_shape(rows, 32 * kblocks));
     if (rows == 0) return MXQ_OK;
     MXQ_TRY(check_ptr(scales, 1));

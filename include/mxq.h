@@ -286,8 +286,9 @@ MXQ_API mxq_status mxq_quantize_mma(mxq_format fmt, const void* src, mxq_dtype d
  * mxq_quantize, mxq_exp_quantize or mxq_quantize_cols for its transposed
  * operand) into the tiled layout. out: device, 4-byte aligned,
  * mxq_mma_scales_bytes(rows, 32 * kblocks) bytes, all written (pad = 0); it
- * may not overlap scales. rows == 0 is a no-op; rows < 0 or kblocks <= 0 ->
- * MXQ_ERR_SHAPE. */
+ * may not overlap scales. rows == 0 is a no-op; rows < 0, kblocks <= 0 or
+ * kblocks > 67108860 (4 * (2^31 - 1) / 128: one tile-row's output words are
+ * counted in 32 bits) -> MXQ_ERR_SHAPE. */
 MXQ_API mxq_status mxq_swizzle_scales(const void* scales, int64_t rows, int64_t kblocks, void* out,
                                       mxq_stream stream);
 

@@ -136,6 +136,10 @@ def test_statuses_before_any_cuda_call(L):
     assert dx(0, 5, None, None, 1, 64, None, 0, None) == 1
     assert fx(5, 3, None, 1, 1 << 40, 1 << 20, None, None) == 2
     assert fx(5, 3, None, 1, 1, 64, None, None) == 1
+    sw = mxq.mxq_swizzle_scales
+    assert sw(None, 8, 4 * (0x7FFFFFFF // 128) + 1, None, None) == 2  # one tile-row's words beyond 32 bits
+    assert sw(None, 8, 0, None, None) == 2 and sw(None, -1, 4, None, None) == 2
+    assert sw(None, 0, 4, None, None) == 0
     assert mxq.mxq_selftest_timeout(0) == 1 and mxq.mxq_selftest_timeout(1001) == 1
     for s in range(7):
         assert mxq.mxq_status_string(s)

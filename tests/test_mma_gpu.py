@@ -59,7 +59,8 @@ def test_quantize_mma_matches_oracle(fmt, dtype, shape):
     assert np.array_equal(scales.cpu().numpy(), want_tiled)
 
 
-@pytest.mark.parametrize("rows,kb", [(1, 1), (3, 5), (127, 3), (128, 4), (129, 9), (1000, 33), (4096, 128)])
+@pytest.mark.parametrize("rows,kb", [(1, 1), (3, 5), (127, 3), (128, 4), (129, 9), (1000, 33), (4096, 128),
+                                     (16384, 256), (300, 1028)])
 def test_swizzle_scales_matches_oracle(rows, kb):
     s = np.asarray(synthetic.uniform_ints(rows + 17 * kb, 3, rows * kb, 256), dtype=np.uint8).reshape(rows, kb)
     out = torch.full((mxq.mxq_mma_scales_bytes(rows, 32 * kb),), 0xEE, dtype=torch.uint8, device="cuda")
