@@ -90,9 +90,42 @@ __device__ __forceinline__ uint32_t code_pair(const uint32_t* w, int i, float in
     }
 }
 
+// AXS-6 codes of the two bf16 values of word w (low half first), g2 = 2^(4 - Es) in both bf16
+// lanes: |x| * 2^(4 - Es) = 16|y| is exact, and one bf16x2 fused multiply-add with 192 rounds it
+// to an integer, ties to even (bf16's unit in the last place is 1 on [128, 256) and 16|y| < 32),
+// so each lane holds 192 + rne(16|y|); minus 192, clamped at 31 by a 16x2 minimum, the sign
+// copied from bit 15 of each lane. Returns code_lo | code_hi << 6.
+__device__ __forceinline__ uint32_t axs6_pair_bf16(uint32_t w, uint32_t g2) {
+    uint32_t t, m2;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(t) : "r"(w & 0x7FFF7FFFu), "r"(g2), "r"(0x43404340u));
+    asm("min.u16x2 %0, %1, %2;" : "=r"(m2) : "r"(t - 0x43404340u), "r"(0x001F001Fu));
+    const uint32_t c2 = m2 | ((w >> 10) & 0x00200020u);
+    return c2 - (c2 >> 16) * 65472u;
+}
+
+// the four 12-bit pairs of codes q[0..3] (eight 6-bit codes) -> three payload words
+__device__ __forceinline__ void pack6x8(const uint32_t* q, uint32_t* out) {
+    out[0] = q[0] | (q[1] << 24);
+    out[1] = (q[1] >> 8) | (q[2] << 16);
+    out[2] = (q[2] >> 16) | (q[3] << 8);
+}
+
 // payload words of a block (P/4 of them: 6-bit 6, E4M3 8, E2M1 4)
 template <int F, typename T>
 __device__ __forceinline__ void encode_block(const uint32_t* w, uint32_t byte, uint32_t* out) {
+    if constexpr (F == F_AXS6 && sizeof(T) == 2) {
+        // bf16 values, scale 2^(4 - Es) a normal bf16 (scale bytes 4 .. 254): two values per word
+        if (byte >= 4u && byte <= 254u) {
+            const uint32_t g = (258u - byte) << 7;
+            const uint32_t g2 = g | (g << 16);
+            uint32_t z[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) z[j] = axs6_pair_bf16(w[2 * j], g2) | (axs6_pair_bf16(w[2 * j + 1], g2) << 12);
+            pack6x8(z, out);
+            pack6x8(z + 4, out + 3);
+            return;
+        }
+    }
     const float inv = inv_scale(byte);
     const uint32_t keep = byte == 0xFFu ? 0u : 0xFFFFFFFFu;
     if constexpr (Fmt<F>::W == 6) {
