@@ -115,7 +115,36 @@ __device__ __forceinline__ void exp_quant_block(uint32_t (&w)[32], float mr, lon
     pm = max3_nan(pm, q[9], q[10]);  // p >= 0 or NaN: the block maximum (or NaN)
     const uint32_t byte = scale_byte<F>(__float_as_uint(pm) & 0x7FFFFFFFu);
     uint32_t out[8];
-    encode_block<F, float>(w, byte, out);
+    if constexpr (F == F_AXS6) {
+        // probabilities are never negative: m = min(rne(p * 2^(4 - Es)), 31) by one packed
+        // fused multiply-add with 1.5 * 2^23 per pair (the product is exact, the add rounds it
+        // to an integer, ties to even), no sign to carry; scale bytes 4 .. 254 (2^(4 - Es) a
+        // normal fp32), the rest (and NaN blocks) through the general encoder
+        if (byte >= 4u && byte <= 254u) {
+            const unsigned long long G = dup2(__uint_as_float((258u - byte) << 23)), C = dup2(kRound);
+            uint32_t z[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                uint32_t c[2];
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    float ta, tb;
+                    upk(f2fma(pk(__uint_as_float(w[4 * j + 2 * q]), __uint_as_float(w[4 * j + 2 * q + 1])), G, C), ta, tb);
+                    uint32_t m2;
+                    asm("min.u16x2 %0, %1, %2;" : "=r"(m2) : "r"(__byte_perm(__float_as_uint(ta), __float_as_uint(tb), 0x5410)),
+                        "r"(0x001F001Fu));
+                    c[q] = m2 - (m2 >> 16) * 65472u;  // code_lo | code_hi << 6
+                }
+                z[j] = c[0] | (c[1] << 12);
+            }
+            pack6x8(z, out);
+            pack6x8(z + 4, out + 3);
+        } else {
+            encode_block<F, float>(w, byte, out);
+        }
+    } else {
+        encode_block<F, float>(w, byte, out);
+    }
     store_payload<F>(codes, blk, out, a32);
     store_scale<F>(scales, blk, byte);
 }
