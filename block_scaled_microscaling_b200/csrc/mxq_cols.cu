@@ -489,16 +489,19 @@ template <int F> __device__ __forceinline__ bool half_has_nan(const uint32_t* hw
 // 8-byte cp.async copies into a ring of three stages, the scales by plain loads into a register
 // that is written to its stage one iteration later. cp.async waits are the hardware's own (no
 // spin on a flag), so no wait here needs a bound.
-// Decode: warp w takes row-blocks (w & 3) and (w & 3) + 4 of column group w >> 2 (32 columns);
-// lane L columns 2p, 2p + 1 of the group (p = L & 15), rows 16h .. 16h + 15 of each row-block
-// (h = L >> 4), so each decoded word is one row's pair of neighbouring columns.
-constexpr int kDqCols = 64, kDqRbt = 8, kDqRows = 32 * kDqRbt, kDqStages = 3;
+// Decode, bf16 output (64 columns): warp w takes row-blocks (w & 3) and (w & 3) + 4 of column
+// group w >> 2 (32 columns); lane L columns 2p, 2p + 1 of the group (p = L & 15), rows 16h ..
+// 16h + 15 of each row-block (h = L >> 4), so each decoded word is one row's pair of neighbouring
+// columns. fp32 output (32 columns): warp w takes row-block w, lane j column j (a whole block),
+// each decoded value one word of its row.
+constexpr int kDqRbt = 8, kDqRows = 32 * kDqRbt, kDqStages = 3;
+template <typename T> __host__ __device__ constexpr int dq_cols() { return 128 / (int)sizeof(T); }  // columns of a tile
 
-template <int F> struct DqStage {
+template <int F, int NC> struct DqStage {
     static constexpr int PB = payload<F>(), SB = Fmt<F>::FIXED ? 2 : 1;
     static constexpr int CS = kDqRbt * PB + 8;                      // padded column stride of the payloads
-    static constexpr int SC = kDqCols * CS;                          // offset of the scales
-    static constexpr int bytes = (SC + kDqCols * kDqRbt * SB + 15) / 16 * 16;
+    static constexpr int SC = NC * CS;                               // offset of the scales
+    static constexpr int bytes = (SC + NC * kDqRbt * SB + 15) / 16 * 16;
 };
 
 __device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
@@ -551,11 +554,12 @@ template <int F> __device__ __forceinline__ void dq_vals16(const uint32_t* hw, f
 
 // Sizes: every byte offset into the codes, scales and output fits in 31 bits (the launcher
 // checks), so the per-tile arithmetic is 32-bit.
-template <int F>
-__global__ void __launch_bounds__(kColThreads, 2) k_dequantize_cols_bf16(const void* __restrict__ codes,
-                                                                        const void* __restrict__ scales,
-                                                                        void* __restrict__ dst, int rows, int cols) {
-    using St = DqStage<F>;
+template <int F, typename T>
+__global__ void __launch_bounds__(kColThreads, 2) k_dequantize_cols_p(const void* __restrict__ codes,
+                                                                     const void* __restrict__ scales,
+                                                                     void* __restrict__ dst, int rows, int cols) {
+    constexpr int kDqCols = dq_cols<T>();
+    using St = DqStage<F, kDqCols>;
     constexpr int PB = St::PB, SB = St::SB, CS = St::CS;
     constexpr int SEG8 = kDqRbt * PB / 8;             // 8-byte pieces of one column's payloads in a tile
     constexpr int NU = kDqCols * SEG8 / kColThreads;  // this thread's pieces of a full tile
@@ -567,7 +571,7 @@ __global__ void __launch_bounds__(kColThreads, 2) k_dequantize_cols_bf16(const v
     const int RB = rows / 32;
     const int nby = (rows + kDqRows - 1) / kDqRows;
     const int ntx = (cols + kDqCols - 1) / kDqCols;
-    const bool a32 = ((reinterpret_cast<uintptr_t>(dst) | (uintptr_t)(cols * 2)) & 31) == 0;
+    const bool a32 = ((reinterpret_cast<uintptr_t>(dst) | (uintptr_t)(cols * sizeof(T))) & 31) == 0;
     const uint32_t st0 = smem_u32(stages);
     const int col_bytes = RB * PB;  // one column's payloads in the transposed layout
     // a column's scales of a full tile are one aligned 8-byte (AXS-6: 16-byte) load when the
@@ -644,22 +648,28 @@ __global__ void __launch_bounds__(kColThreads, 2) k_dequantize_cols_bf16(const v
         else *reinterpret_cast<uint2*>(stages + soff) = make_uint2(sw.x, sw.y);
     };
 
-    // decode role: row-blocks rb and rb + 4 of column group cg; columns ja, ja + 1, rows 16h ..
-    const int rb = warp & 3, cg = warp >> 2;
+    // decode role (bf16): row-blocks rb and rb + 4 of column group cg; columns ja, ja + 1, rows 16h ..
+    const int rb = sizeof(T) == 2 ? (warp & 3) : warp, cg = sizeof(T) == 2 ? (warp >> 2) : 0;
     const int p = lane & 15, h = lane >> 4;
-    const int ja = cg * 32 + 2 * p;
+    const int ja = sizeof(T) == 2 ? cg * 32 + 2 * p : lane;
     const int pa_off = ja * CS + rb * PB, sa_off = St::SC + (ja * kDqRbt + rb) * SB;
-    uint8_t* const obase = tile + (rb * 32 + 16 * h) * 128 + 4 * (p & 3);
-    uint32_t c16[4];
+    uint8_t* const obase = sizeof(T) == 2 ? tile + (rb * 32 + 16 * h) * 128 + 4 * (p & 3)
+                                          : tile + rb * 32 * 128 + 4 * (lane & 3);
+    uint32_t c16[8];  // bf16: chunk offsets by row & 3 (4 used); fp32: by row & 7
 #pragma unroll
-    for (int q = 0; q < 4; ++q) c16[q] = (uint32_t)(16 * ((4 * cg + (p >> 2)) ^ dq_swz(q + 16 * h)));
-    // store role: thread (r, hf) stores bytes 32hf .. 32hf + 31 of output rows r and r + 128 and,
-    // in a full 64-column strip, bytes 64 + 32hf .. (a strip of 32 columns is 64 bytes)
-    const int r = t >> 1, hf = t & 1;
-    uint32_t rd[4];  // byte offsets of its four chunks of row r in the output tile (row r + 128: + 128 * 128)
+    for (int q = 0; q < 8; ++q)
+        c16[q] = sizeof(T) == 2 ? (uint32_t)(16 * ((4 * cg + (p >> 2)) ^ dq_swz((q & 3) + 16 * h)))
+                                : (uint32_t)(16 * ((lane >> 2) ^ q));
+    // store role, bf16: thread (r, hf) stores bytes 32hf .. 32hf + 31 of output rows r and r + 128
+    // and, in a full 64-column strip, bytes 64 + 32hf .. (a strip of 32 columns is 64 bytes);
+    // fp32: thread t stores its row t, 128 bytes (chunk c at c ^ (t & 7))
+    const int r = sizeof(T) == 2 ? (t >> 1) : t, hf = sizeof(T) == 2 ? (t & 1) : 0;
+    uint32_t rd[8];  // byte offsets of its chunks in the output tile (bf16: 4 of row r; row r + 128: + 128 * 128)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) rd[c] = (uint32_t)(r * 128 + 16 * (((c & 1) + 2 * hf + 4 * (c >> 1)) ^ dq_swz(r)));
-    const int rowoff = r * cols * 2 + 32 * hf;
+    for (int c = 0; c < 8; ++c)
+        rd[c] = sizeof(T) == 2 ? (uint32_t)(r * 128 + 16 * ((((c & 3) & 1) + 2 * hf + 4 * ((c & 3) >> 1)) ^ dq_swz(r)))
+                               : (uint32_t)(r * 128 + 16 * (c ^ (r & 7)));
+    const int rowoff = r * cols * (int)sizeof(T) + 32 * hf;
 
     DqWalk cur(ntx, nby), ahead(ntx, nby);
     int so = -1;
@@ -675,73 +685,129 @@ __global__ void __launch_bounds__(kColThreads, 2) k_dequantize_cols_bf16(const v
         cp_async_wait<1>();  // this thread's copies of the tile have landed
         __syncthreads();     // everyone's have; the previous tile's rows have left the output tile
         const uint8_t* stg = stages + stage * St::bytes;
-        if (cg * 32 < ncols) {
+        if constexpr (sizeof(T) == 2) {
+            if (cg * 32 < ncols) {
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                if (rb + 4 * half >= nrows / 32) break;
-                const uint8_t* sp = stg + pa_off + half * 4 * PB;
-                uint32_t ha[Fmt<F>::W / 2], hb[Fmt<F>::W / 2];
-                load_half_payload<F>(sp, h, ha);
-                load_half_payload<F>(sp + CS, h, hb);
-                uint32_t ba, bb;
-                if constexpr (SB == 2) {
-                    ba = *reinterpret_cast<const uint16_t*>(stg + sa_off + half * 4 * SB) & 0xFFu;
-                    bb = *reinterpret_cast<const uint16_t*>(stg + sa_off + half * 4 * SB + kDqRbt * SB) & 0xFFu;
-                } else {
-                    ba = stg[sa_off + half * 4];
-                    bb = stg[sa_off + half * 4 + kDqRbt];
+                for (int half = 0; half < 2; ++half) {
+                    if (rb + 4 * half >= nrows / 32) break;
+                    const uint8_t* sp = stg + pa_off + half * 4 * PB;
+                    uint32_t ha[Fmt<F>::W / 2], hb[Fmt<F>::W / 2];
+                    load_half_payload<F>(sp, h, ha);
+                    load_half_payload<F>(sp + CS, h, hb);
+                    uint32_t ba, bb;
+                    if constexpr (SB == 2) {
+                        ba = *reinterpret_cast<const uint16_t*>(stg + sa_off + half * 4 * SB) & 0xFFu;
+                        bb = *reinterpret_cast<const uint16_t*>(stg + sa_off + half * 4 * SB + kDqRbt * SB) & 0xFFu;
+                    } else {
+                        ba = stg[sa_off + half * 4];
+                        bb = stg[sa_off + half * 4 + kDqRbt];
+                    }
+                    float va[16], vb[16];
+                    dq_vals16<F>(ha, va);
+                    dq_vals16<F>(hb, vb);
+                    const unsigned long long S = pk(fwd_scale(ba), fwd_scale(bb));
+                    uint32_t o[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        float x, y;
+                        upk(f2mul(pk(va[k], vb[k]), S), x, y);
+                        o[k] = bf16x2(x, y);
+                    }
+                    if (ba == 0xFFu || bb == 0xFFu || half_has_nan<F>(ha) || half_has_nan<F>(hb)) {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {  // canonical quiet NaN for NaN blocks and E4M3 NaN codes
+                            const bool na = ba == 0xFFu || (F == F_E4M3 && ((ha[k >> 2] >> (8 * (k & 3))) & 0x7Fu) == 0x7Fu);
+                            const bool nb = bb == 0xFFu || (F == F_E4M3 && ((hb[k >> 2] >> (8 * (k & 3))) & 0x7Fu) == 0x7Fu);
+                            if (na) o[k] = (o[k] & 0xFFFF0000u) | 0x7FC0u;
+                            if (nb) o[k] = (o[k] & 0x0000FFFFu) | 0x7FC00000u;
+                        }
+                    }
+                    uint8_t* ob = obase + half * 128 * 128;  // row-block rb + 4: 128 rows further
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) *reinterpret_cast<uint32_t*>(ob + k * 128 + c16[k & 3]) = o[k];
                 }
-                float va[16], vb[16];
-                dq_vals16<F>(ha, va);
-                dq_vals16<F>(hb, vb);
-                const unsigned long long S = pk(fwd_scale(ba), fwd_scale(bb));
-                uint32_t o[16];
+            }
+        } else {
+            if (rb < nrows / 32) {  // one row-block per warp, lane j = column j, all 32 rows
+                const uint8_t* sp = stg + pa_off;
+                uint32_t ha[Fmt<F>::W / 2], hb[Fmt<F>::W / 2];
+                load_half_payload<F>(sp, 0, ha);
+                load_half_payload<F>(sp, 1, hb);
+                const uint32_t byte =
+                    SB == 2 ? (*reinterpret_cast<const uint16_t*>(stg + sa_off) & 0xFFu) : (uint32_t)stg[sa_off];
+                float v[32];
+                dq_vals16<F>(ha, v);
+                dq_vals16<F>(hb, v + 16);
+                const unsigned long long S = dup2(fwd_scale(byte));
+                uint32_t o[32];
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
                     float x, y;
-                    upk(f2mul(pk(va[k], vb[k]), S), x, y);
-                    o[k] = bf16x2(x, y);
+                    upk(f2mul(pk(v[2 * k], v[2 * k + 1]), S), x, y);
+                    o[2 * k] = __float_as_uint(x);
+                    o[2 * k + 1] = __float_as_uint(y);
                 }
-                if (ba == 0xFFu || bb == 0xFFu || half_has_nan<F>(ha) || half_has_nan<F>(hb)) {
+                if (byte == 0xFFu || half_has_nan<F>(ha) || half_has_nan<F>(hb)) {
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) {  // canonical quiet NaN for NaN blocks and E4M3 NaN codes
-                        const bool na = ba == 0xFFu || (F == F_E4M3 && ((ha[k >> 2] >> (8 * (k & 3))) & 0x7Fu) == 0x7Fu);
-                        const bool nb = bb == 0xFFu || (F == F_E4M3 && ((hb[k >> 2] >> (8 * (k & 3))) & 0x7Fu) == 0x7Fu);
-                        if (na) o[k] = (o[k] & 0xFFFF0000u) | 0x7FC0u;
-                        if (nb) o[k] = (o[k] & 0x0000FFFFu) | 0x7FC00000u;
+                    for (int k = 0; k < 32; ++k) {  // canonical quiet NaN for NaN blocks and E4M3 NaN codes
+                        const uint32_t* hw = k < 16 ? ha : hb;
+                        const int kk = k & 15;
+                        if (byte == 0xFFu || (F == F_E4M3 && ((hw[kk >> 2] >> (8 * (kk & 3))) & 0x7Fu) == 0x7Fu))
+                            o[k] = 0x7FC00000u;
                     }
                 }
-                uint8_t* ob = obase + half * 128 * 128;  // row-block rb + 4: 128 rows further
 #pragma unroll
-                for (int k = 0; k < 16; ++k) *reinterpret_cast<uint32_t*>(ob + k * 128 + c16[k & 3]) = o[k];
+                for (int k = 0; k < 32; ++k) *reinterpret_cast<uint32_t*>(obase + k * 128 + c16[k & 7]) = o[k];
             }
         }
         __syncthreads();  // the output tile is complete; this stage is free
         put_scale(so);    // the next tile's scales into its stage (read after the next barrier)
         issue(ahead, stage == 0 ? kDqStages - 1 : stage - 1, so);
         ahead.next();
+        if constexpr (sizeof(T) == 2) {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            if (r + 128 * half < nrows) {
-                char* q = dbase + ((row0 + 128 * half) * cols + col0) * 2 + rowoff;
-                uint32_t w[16];
+            for (int half = 0; half < 2; ++half) {
+                if (r + 128 * half < nrows) {
+                    char* q = dbase + ((row0 + 128 * half) * cols + col0) * 2 + rowoff;
+                    uint32_t w[16];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(tile + rd[c] + half * 128 * 128);
-                    w[4 * c] = v.x;
-                    w[4 * c + 1] = v.y;
-                    w[4 * c + 2] = v.z;
-                    w[4 * c + 3] = v.w;
+                    for (int c = 0; c < 4; ++c) {
+                        const uint4 v = *reinterpret_cast<const uint4*>(tile + rd[c] + half * 128 * 128);
+                        w[4 * c] = v.x;
+                        w[4 * c + 1] = v.y;
+                        w[4 * c + 2] = v.z;
+                        w[4 * c + 3] = v.w;
+                    }
+                    st32(q, w, a32);
+                    if (ncols == kDqCols) st32(q + 64, w + 8, a32);
                 }
-                st32(q, w, a32);
-                if (ncols == kDqCols) st32(q + 64, w + 8, a32);
+            }
+        } else {
+            if (r < nrows) {
+                char* q = dbase + (row0 * cols + col0) * 4 + rowoff;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const uint4 v = *reinterpret_cast<const uint4*>(tile + rd[4 * hh + c]);
+                        w[4 * c] = v.x;
+                        w[4 * c + 1] = v.y;
+                        w[4 * c + 2] = v.z;
+                        w[4 * c + 3] = v.w;
+                    }
+                    st32(q + 64 * hh, w, a32);
+                    st32(q + 64 * hh + 32, w + 8, a32);
+                }
             }
         }
     }
     cp_async_wait<0>();  // no copy may land in shared memory after the CTA has left
 }
 
-template <int F> static constexpr int dq_bf16_smem() { return kDqRows * 128 + kDqStages * DqStage<F>::bytes; }
+template <int F, typename T> static constexpr int dq_p_smem() {
+    return kDqRows * 128 + kDqStages * DqStage<F, dq_cols<T>()>::bytes;
+}
 
 template <int F, typename T>
 static cudaError_t launch_qc_t(const void* src, void* codes, void* scales, long long rows, long long cols,
@@ -773,28 +839,27 @@ static cudaError_t launch_qc_t(const void* src, void* codes, void* scales, long 
 template <int F, typename T>
 static cudaError_t launch_dqc_t(const void* codes, const void* scales, void* dst, long long rows, long long cols,
                                 cudaStream_t st) {
-    if constexpr (sizeof(T) == 2) {
-        // 32-bit offsets: the outputs, the codes and the scales each below 2^31 bytes
-        if (rows * cols * 2 < (1LL << 31) && rows * (cols / 32) * payload<F>() < (1LL << 31)) {
-            auto kern = k_dequantize_cols_bf16<F>;
-            constexpr int smem = dq_bf16_smem<F>();
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (e != cudaSuccess) return e;
-            int dev = 0, sms = 148, per_sm = 1;
-            cudaGetDevice(&dev);
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kColThreads, smem);
-            // two CTAs per SM, though shared memory would hold three: the 8-byte copies are staged
-            // through L1, and a third CTA's stages leave L1 too small for them (bf16 16384x8192,
-            // fraction of the HBM peak, E2M3 / E4M3 / E2M1: 0.57 / 0.90 / 0.80 with three CTAs,
-            // 0.81 / 0.92 / 0.84 with two)
-            if (per_sm > 2) per_sm = 2;
-            const long long ntiles = ((cols + kDqCols - 1) / kDqCols) * ((rows + kDqRows - 1) / kDqRows);
-            long long grid = (long long)sms * (per_sm > 0 ? per_sm : 1);
-            if (grid > ntiles) grid = ntiles;
-            kern<<<(unsigned)grid, kColThreads, smem, st>>>(codes, scales, dst, (int)rows, (int)cols);
-            return cudaGetLastError();
-        }
+    // 32-bit offsets: the outputs, the codes and the scales each below 2^31 bytes
+    if (rows * cols * (long long)sizeof(T) < (1LL << 31) && rows * (cols / 32) * payload<F>() < (1LL << 31)) {
+        auto kern = k_dequantize_cols_p<F, T>;
+        constexpr int smem = dq_p_smem<F, T>();
+        constexpr int NC = dq_cols<T>();
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        int dev = 0, sms = 148, per_sm = 1;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kColThreads, smem);
+        // two CTAs per SM, though shared memory would hold three: the 8-byte copies are staged
+        // through L1, and a third CTA's stages leave L1 too small for them (bf16 16384x8192,
+        // fraction of the HBM peak, E2M3 / E4M3 / E2M1: 0.57 / 0.90 / 0.80 with three CTAs,
+        // 0.81 / 0.92 / 0.84 with two)
+        if (per_sm > 2) per_sm = 2;
+        const long long ntiles = ((cols + NC - 1) / NC) * ((rows + kDqRows - 1) / kDqRows);
+        long long grid = (long long)sms * (per_sm > 0 ? per_sm : 1);
+        if (grid > ntiles) grid = ntiles;
+        kern<<<(unsigned)grid, kColThreads, smem, st>>>(codes, scales, dst, (int)rows, (int)cols);
+        return cudaGetLastError();
     }
     dim3 grid((unsigned)(cols / kNarrowCols), (unsigned)((rows + kTileRows - 1) / kTileRows));
     k_dequantize_cols<F, T><<<grid, kColThreads, 0, st>>>(codes, scales, dst, rows, cols);
