@@ -637,7 +637,7 @@ PROFILE_CASES = ["batch_weight", "q_e2m3_weight", "q_e3m2_weight", "dq_e2m3_weig
                  "q_e2m3_layer", "fq_axs6_grad", "exp_mxfp4_scores", "expfree_mxfp4_scores", "qcols_e2m3_weight",
                  "dqcols_e2m3_weight", "qcols_e2m3_act", "dqcols_e2m3_act", "exmy_e3m3_act", "dq_exmy_e3m3_act",
                  "fq_exmy_e3m3_act", "qmma_mxfp8_act", "dq_e2m3_act", "fq_axs6_quickstart",
-                 "swizzle_scales_act", "exp_e2m3_scores", "exp_axs6_scores"]
+                 "swizzle_scales_act", "exp_e2m3_scores", "exp_axs6_scores", "dqcols_e2m3_f32"]
 
 
 def profile_case(name, reps):
@@ -672,6 +672,11 @@ def profile_case(name, reps):
         y = torch.empty_like(x)
         fn = (lambda: mxq.quantize_cols(x, "mxfp6_e2m3", codes=cc, scales=cs)) if name[0] == "q" else \
             (lambda: mxq.dequantize_cols(cc, cs, "mxfp6_e2m3", x.shape, out=y))
+    elif name == "dqcols_e2m3_f32":
+        x = torch.randn(8192, 8192, device=dev, generator=gen) * 0.02
+        cc, cs = mxq.quantize_cols(x, "mxfp6_e2m3")
+        y = torch.empty_like(x)
+        fn = lambda: mxq.dequantize_cols(cc, cs, "mxfp6_e2m3", x.shape, out=y)
     elif name == "dq_e2m3_act":
         x = (torch.randn(16384, 8192, device=dev, generator=gen) * 0.5).to(torch.bfloat16)
         c, s = mxq.quantize(x, "mxfp6_e2m3")
