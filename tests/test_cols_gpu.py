@@ -124,3 +124,55 @@ def test_cols_large_sampled_columns(fmt, dtype, shape):
     out = mxq.dequantize_cols(codes, scales, fmt, (rows, cols), tdtype(dtype))
     ref = oracle.dequantize(oc, os_, fmt, xs.shape, dtype)
     assert np.array_equal(bits(host(out)[:, sel].T.copy()), bits(ref))
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("dtype,shape", [("bf16", (4192, 4128)), ("f32", (2336, 4160))])
+def test_dequantize_cols_random_codes(fmt, dtype, shape):
+    """Every code value (E4M3 NaN codes included) and every scale byte (0 and 0xFF included) in the
+    transposed layout, at a ragged multi-tile size: dequantize_cols equals the oracle's dequantize
+    of the same codes, transposed back."""
+    rows, cols = shape
+    assert_walks_several_tiles(rows, cols, dtype)
+    rng = np.random.default_rng(zlib.crc32(repr(("rnd", fmt, dtype, shape)).encode()))
+    pb = oracle.payload_bytes(fmt)
+    codes = rng.integers(0, 256, (cols, rows // 32 * pb), dtype=np.uint8)
+    sb = rng.integers(0, 256, (cols, rows // 32)).astype(np.uint16)
+    sb.reshape(-1)[:256] = np.arange(256)
+    if fmt == "axs6":
+        sb |= (rng.integers(0, 4, sb.shape) << 8).astype(np.uint16)  # config bits are ignored on read
+        scales, tscales = sb, torch.from_numpy(sb.view(np.int16)).cuda()
+    else:
+        scales = sb.astype(np.uint8)
+        tscales = torch.from_numpy(scales).cuda()
+    out = mxq.dequantize_cols(torch.from_numpy(codes).cuda(), tscales, fmt, (rows, cols), tdtype(dtype))
+    ref = np.ascontiguousarray(oracle.dequantize(codes, scales, fmt, (cols, rows), dtype).T)
+    assert np.array_equal(bits(host(out)), bits(ref))
+
+
+@pytest.mark.parametrize("dtype,shape", [("bf16", (2080, 8224)), ("f32", (2336, 4160)), ("bf16", (96, 96))])
+def test_cols_outputs_stay_inside_their_buffers(dtype, shape):
+    """Guard bands: sentinel bytes around the codes, the scales and the values that the column
+    kernels write stay untouched, at shapes with a last row band of one row-block and (bf16) a
+    last column strip of 32 columns."""
+    rows, cols = shape
+    x = big_values(rows, cols, dtype, seed=11)
+    for fmt in FMTS:
+        nc = cols * (rows // 32) * oracle.payload_bytes(fmt)
+        ns = cols * (rows // 32) * (2 if fmt == "axs6" else 1)
+        cbuf = torch.full((nc + 64,), 0xA5, dtype=torch.uint8, device="cuda")
+        sbuf = torch.full((ns + 64,), 0xA5, dtype=torch.uint8, device="cuda")
+        codes = cbuf[32:32 + nc]
+        scales = sbuf[32:32 + ns].view(torch.int16 if fmt == "axs6" else torch.uint8)
+        mxq.quantize_cols(dev(x), fmt, codes=codes, scales=scales, check=True)
+        cb, sbh = host(cbuf), host(sbuf)
+        assert np.all(cb[:32] == 0xA5) and np.all(cb[32 + nc:] == 0xA5)
+        assert np.all(sbh[:32] == 0xA5) and np.all(sbh[32 + ns:] == 0xA5)
+        esz = 4 if dtype == "f32" else 2
+        obuf = torch.full(((rows * cols * esz + 128) // 4,), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
+        ov = obuf.view(torch.uint8)[64:64 + rows * cols * esz].view(tdtype(dtype)).view(rows, cols)
+        mxq.dequantize_cols(codes, scales, fmt, (rows, cols), out=ov)
+        ob = host(obuf.view(torch.uint8))
+        assert np.all(ob[:64] == 0x5A) and np.all(ob[64 + rows * cols * esz:] == 0x5A)
+        ref = oracle.dequantize(host(codes).reshape(cols, -1), host(scales).reshape(cols, -1), fmt, (cols, rows), dtype)
+        assert np.array_equal(bits(host(ov)), bits(np.ascontiguousarray(ref.T)))
