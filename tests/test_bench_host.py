@@ -248,3 +248,23 @@ def test_stack_step_bytes_are_the_survey_figures():
     b, n = bench.stack_step_bytes()
     assert n == 36 * 100925440
     assert b == 36 * (280698880 + 283852800)
+
+
+def test_timed_region_with_a_set_status_word_reports_nothing():
+    """The status check runs after every timed region; when it raises (a bounded wait ran out,
+    so some outputs are incomplete), the exception leaves timed_replay and no time is returned."""
+    t = FakeTorch()
+    g = FakeGraph(t, [12.5, 99.0])
+
+    class Timeout(RuntimeError):
+        pass
+
+    def check():
+        raise Timeout("MXQ_ERR_TIMEOUT")
+
+    with pytest.raises(Timeout):
+        bench.timed_replay(t, g, "cpu", None, sampler_sequence([GOOD, GOOD]), after=check)
+    calls = []
+    ms, _ = bench.timed_replay(t, FakeGraph(t, [3.0, 4.0, 99.0]), "cpu", None, sampler_sequence([GOOD]),
+                               replays=2, after=lambda: calls.append(1))
+    assert ms == 7.0 and calls == [1]  # K replays in one region, one check after it
