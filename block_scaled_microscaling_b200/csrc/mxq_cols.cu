@@ -479,10 +479,11 @@ template <int F> __device__ __forceinline__ bool half_has_nan(const uint32_t* hw
     }
 }
 
-// ---- dequantize to bf16: persistent, payloads prefetched two tiles ahead --------------------------
+// ---- dequantize: persistent, payloads prefetched two tiles ahead ----------------------------------
 //
-// Tiles of 256 rows x 64 columns (128-byte output rows, one whole line per row; a column's 8
-// row-blocks of payload are one 192-byte run on a 64-byte boundary: whole DRAM accesses). Each
+// Tiles of 256 rows x 128 output bytes per row (64 bf16 or 32 fp32 columns: one whole line per
+// row; a column's 8 row-blocks of payload are one run of 8 payloads, 192 bytes for the 6-bit
+// formats, on a 64-byte boundary when the column's run is: whole DRAM accesses). Each
 // CTA walks tiles blockIdx.x + n * gridDim.x in band-major order (the CTAs running at one time
 // cover a few adjacent row bands, so the rows they write are close together) and keeps the loads
 // of tiles n + 1 and n + 2 in flight while it decodes and stores tile n: the payloads come in by
