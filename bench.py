@@ -571,12 +571,13 @@ def workloads_breakdown(torch, mxq, hbm):
         del g
         rec(f"c2_weight_{nm}_bf16", op_bytes, n2, ms)
     # column-direction blocks of the same weight (32 rows of a column), transposed layout: 8 launches
-    # per round on the 8 sets, so each reads data last touched 7 launches (330 MB) earlier
+    # per round on the 8 sets, so each reads data last touched 7 launches (330 MB) earlier; 50
+    # rounds, 400 launches per graph as for the single-operation rows
     ccs = [mxq.quantize_cols(st["x"], "mxfp6_e2m3") for st in sets]
     ts = time_launches(torch, [
         lambda: [mxq.quantize_cols(st["x"], "mxfp6_e2m3", codes=c, scales=sc_) for st, (c, sc_) in zip(sets, ccs)],
         lambda: [mxq.dequantize_cols(c, sc_, "mxfp6_e2m3", st["x"].shape, out=st["ya"])
-                 for st, (c, sc_) in zip(sets, ccs)]], 2)
+                 for st, (c, sc_) in zip(sets, ccs)]], 50)
     rec("c2_weight_quantize_cols_e2m3_bf16", op_bytes, n2, ts[0] / len(sets))
     rec("c2_weight_dequantize_cols_e2m3_bf16", op_bytes, n2, ts[1] / len(sets))
     del sets, ccs, w
