@@ -638,7 +638,7 @@ PROFILE_CASES = ["batch_weight", "q_e2m3_weight", "q_e3m2_weight", "dq_e2m3_weig
                  "q_e2m3_layer", "fq_axs6_grad", "exp_mxfp4_scores", "expfree_mxfp4_scores", "qcols_e2m3_weight",
                  "dqcols_e2m3_weight", "qcols_e2m3_act", "dqcols_e2m3_act", "exmy_e3m3_act", "dq_exmy_e3m3_act",
                  "fq_exmy_e3m3_act", "qmma_mxfp8_act", "dq_e2m3_act", "fq_axs6_quickstart",
-                 "swizzle_scales_act", "exp_e2m3_scores", "exp_axs6_scores", "dqcols_e2m3_f32"]
+                 "swizzle_scales_act", "exp_e2m3_scores", "exp_axs6_scores", "dqcols_e2m3_f32", "stack_steady"]
 
 
 def profile_case(name, reps):
@@ -723,6 +723,20 @@ def profile_case(name, reps):
               for _, r, c_ in synthetic.DECODER_LAYER]
         outs = mxq.quantize_grouped(ws, fmt)
         fn = lambda: mxq.quantize_grouped(ws, fmt, outs=outs)
+    elif name == "stack_steady":
+        # three decoder layers; launch k converts layer k mod 3 to E2M3 (k even) or AXS-6 (k odd),
+        # so every launch reads a layer last read three launches (about 850 MB of traffic) earlier
+        # and the previous launch's outputs leave L2 during it, as in the timed step: the DRAM
+        # counters of one launch then hold its whole traffic (no flush between launches)
+        layers = [[(torch.randn(r, c_, device=dev, generator=gen) * 0.02).to(torch.bfloat16)
+                   for _, r, c_ in synthetic.DECODER_LAYER] for _ in range(3)]
+        outs = {f: [mxq.quantize_grouped(ws, f) for ws in layers] for f in STACK_FORMATS}
+        k = [0]
+
+        def fn():
+            f = STACK_FORMATS[k[0] % 2]
+            mxq.quantize_grouped(layers[k[0] % 3], f, outs=outs[f][k[0] % 3])
+            k[0] += 1
     elif name == "fq_axs6_grad":
         g = torch.randn(16384, 8192, device=dev, generator=gen) * 1e-3
         o = torch.empty_like(g)
