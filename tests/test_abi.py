@@ -1,7 +1,6 @@
 """The C ABI library loads and exports every symbol include/mxq.h declares;
 host-only behaviour (size queries, statuses returned before any CUDA call).
 No kernel runs here."""
-import ctypes
 import os
 import re
 import subprocess
