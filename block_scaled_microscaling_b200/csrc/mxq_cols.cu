@@ -340,10 +340,10 @@ static bool encode_tile_map(CUtensorMap* m, const void* base, long long rows, lo
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// ---- dequantize: 32-column tiles (64-byte bf16 rows) -------------------------------------------
-// The 128-byte-row tile above was slower for dequantize (bf16 16384x8192: 0.53 vs 0.62 of the
-// HBM peak), so dequantize keeps tiles of 256 rows x 32 columns, chunk c of row r at c ^ (r/2 mod 4)
-// for 64-byte rows and c ^ (r mod 8) for 128-byte rows.
+// ---- dequantize, one CTA per tile: 32-column tiles (64-byte bf16 rows) ---------------------------
+// Taken only by matrices whose output, codes or scales reach 2^31 bytes (its offsets are 64-bit);
+// the persistent kernel further below takes everything else. Tiles of 256 rows x 32 columns,
+// chunk c of row r at c ^ (r/2 mod 4) for 64-byte rows and c ^ (r mod 8) for 128-byte rows.
 constexpr int kNarrowCols = 32;
 
 // byte offset of element (r, j) of the tile; rows of 32 * sizeof(T) bytes,

@@ -176,3 +176,36 @@ def test_cols_outputs_stay_inside_their_buffers(dtype, shape):
         assert np.all(ob[:64] == 0x5A) and np.all(ob[64 + rows * cols * esz:] == 0x5A)
         ref = oracle.dequantize(host(codes).reshape(cols, -1), host(scales).reshape(cols, -1), fmt, (cols, rows), dtype)
         assert np.array_equal(bits(host(ov)), bits(np.ascontiguousarray(ref.T)))
+
+
+@pytest.mark.parametrize("fmt,dtype,shape", [("mxfp6_e2m3", "f32", (16384, 32768)), ("axs6", "f32", (16384, 32768)),
+                                             ("mxfp8", "bf16", (32768, 32768))])
+def test_dequantize_cols_beyond_31_bit_offsets(fmt, dtype, shape):
+    """A 2 GiB output (2^31 bytes) leaves the persistent dequantize's 32-bit offsets, so the
+    launcher takes the one-CTA-per-tile kernel with 64-bit offsets: the whole matrix converted
+    there and back, 24 sampled columns (the first and last included) compared in full with the
+    oracle. The values come from the device generator (per-column-block exponents over +-30
+    binades, zero and NaN column blocks) and are copied back for the oracle."""
+    rows, cols = shape
+    esz = 4 if dtype == "f32" else 2
+    assert rows * cols * esz >= 1 << 31
+    g = torch.Generator(device="cuda").manual_seed(zlib.crc32(repr(("wide", fmt, dtype, shape)).encode()))
+    x = torch.randn(rows // 32, 32, cols, device="cuda", generator=g)
+    x *= torch.exp2(torch.randint(-30, 31, (rows // 32, 1, cols), device="cuda", generator=g).float())
+    kind = torch.randint(0, 64, (rows // 32, 1, cols), device="cuda", generator=g)
+    x = torch.where(kind == 0, torch.zeros_like(x), x)
+    x[:, 5:6, :] = torch.where(kind == 1, torch.full_like(x[:, 5:6, :], float("nan")), x[:, 5:6, :])
+    x = x.reshape(rows, cols).to(tdtype(dtype))
+    del kind
+    codes, scales = mxq.quantize_cols(x, fmt)
+    rng = np.random.default_rng(7)
+    sel = np.unique(np.concatenate([rng.choice(cols, 22, replace=False), [0, cols - 1]]))
+    xs = np.ascontiguousarray(host(x[:, torch.from_numpy(sel).cuda()]).T)
+    oc, os_ = oracle.quantize(xs, fmt)
+    assert np.array_equal(host(scales[torch.from_numpy(sel).cuda()]), os_)
+    assert np.array_equal(host(codes[torch.from_numpy(sel).cuda()]), oc)
+    del x
+    torch.cuda.empty_cache()
+    out = mxq.dequantize_cols(codes, scales, fmt, (rows, cols), tdtype(dtype))
+    ref = oracle.dequantize(oc, os_, fmt, xs.shape, dtype)
+    assert np.array_equal(bits(host(out[:, torch.from_numpy(sel).cuda()]).T.copy()), bits(ref))
