@@ -858,6 +858,8 @@ def main():
                      "achieved": round(ach, 1), "peak": hbm, "peak_source": how, "unit": "GB/s",
                      "frac": round(ach / hbm, 4), "peak_nominal": NOMINAL_HBM,
                      "frac_nominal": round(ach / NOMINAL_HBM, 4), "traffic": ncu_traffic("grouped_layer"),
+                     "traffic_source": "DRAM bytes read + written per launch, ncu in the step's steady state "
+                                       "(profiles/k_quantize_grouped_decoder_layer_steady_traffic.md)",
                      "algorithmic_bytes_per_launch": int(bytes_per_launch),
                      "launch_ms": round(ms_step / launches_per_step, 5)},
         "clocks": clocks,
